@@ -1,0 +1,142 @@
+"""PrismSparseAttention: the whole forward/backward path through the C ABI.
+
+PyTorch only allocates device memory and supplies the stream; each step is
+one call into libprism_b200.so:
+
+  forward : zone_indicator(V) -> assign_blocks -> permute(Q, K, V) (+ block
+            pooling of Q, K) -> block_select -> bsa_fwd -> unpermute(O)
+  backward: permute(dO) -> bsa_bwd -> unpermute(dQ, dK, dV)
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import prism as P
+
+
+class PrismSparseAttention:
+    """Dynamic block-sparse self-attention over a T x H x W token grid.
+
+    Inputs are natural-layout [N, heads, head_dim] tensors (bf16, or f32 which
+    the permutation rounds to bf16), N = T*H*W in raster order (t, y, x).
+    ``col_capacity`` bounds the number of selected (query block, key block)
+    pairs over all heads; the default allows a quarter of all pairs.
+    ``select_ws_bytes`` bounds the block-score workspace (heads are processed
+    in passes that fit).
+    """
+
+    def __init__(self, T, H, W, heads, head_dim, top_k, top_p, *, tau128=0.5, tau256=0.25, eps=1e-4,
+                 scale=0.0, col_capacity=None, select_ws_bytes=4 << 30, device="cuda"):
+        self.p = P.make_params(T, H, W, heads, head_dim, top_k, top_p, tau128, tau256, eps, scale)
+        self.T, self.H, self.W, self.heads, self.D = T, H, W, heads, head_dim
+        self.N = T * H * W
+        self.Z = self.N // 512
+        self.cap = 8 * self.Z
+        dev = torch.device(device)
+        self.device = dev
+        i32, f32, bf16 = torch.int32, torch.float32, torch.bfloat16
+        Z, cap, N, D = self.Z, self.cap, self.N, head_dim
+        self.g = torch.empty(Z, 3, dtype=f32, device=dev)
+        self.rho = torch.empty(Z, dtype=f32, device=dev)
+        self.debug = torch.empty(Z, 8, dtype=f32, device=dev)
+        self.shape_id = torch.empty(Z, dtype=torch.uint8, device=dev)
+        self.zone_blk_base = torch.empty(Z + 1, dtype=i32, device=dev)
+        self.blocks = torch.empty(cap, 4, dtype=i32, device=dev)
+        self.nblk = torch.empty(1, dtype=i32, device=dev)
+        self.qp = torch.empty(heads, N, D, dtype=bf16, device=dev)
+        self.kp = torch.empty_like(self.qp)
+        self.vp = torch.empty_like(self.qp)
+        self.op = torch.empty_like(self.qp)
+        self.qbar = torch.empty(heads, cap, D, dtype=f32, device=dev)
+        self.kbar = torch.empty_like(self.qbar)
+        self.lse = torch.empty(heads, N, dtype=f32, device=dev)
+        self.row_ptr = torch.empty(heads * cap + 1, dtype=i32, device=dev)
+        if col_capacity is None:
+            col_capacity = min(heads * cap * cap // 4, 2**31 - 1)
+        self.col = torch.empty(int(col_capacity), dtype=i32, device=dev)
+        self.nnz = torch.empty(1, dtype=torch.int64, device=dev)
+        ind, _ = P.prism_workspace_size(self.p, P.PRISM_WS_INDICATOR)
+        self.ws_ind = torch.empty(max(ind, 256), dtype=torch.uint8, device=dev)
+        sel_min, sel_all = P.prism_workspace_size(self.p, P.PRISM_WS_SELECT)
+        self.ws_sel = torch.empty(max(sel_min, min(sel_all, select_ws_bytes)), dtype=torch.uint8, device=dev)
+        self._bwd = None
+
+    # -- forward ------------------------------------------------------------
+    def indicator(self, v, audio=None):
+        P.prism_zone_indicator(self.p, v, audio, self.g, self.rho, self.debug, self.ws_ind)
+
+    def assign(self):
+        P.prism_assign_blocks(self.p, self.g, self.rho, self.shape_id, self.zone_blk_base, self.blocks, self.nblk)
+
+    def permute(self, q, k, v):
+        P.prism_permute(self.p, self.shape_id, self.zone_blk_base, q, self.qp, self.qbar)
+        P.prism_permute(self.p, self.shape_id, self.zone_blk_base, k, self.kp, self.kbar)
+        P.prism_permute(self.p, self.shape_id, self.zone_blk_base, v, self.vp, None)
+
+    def select(self):
+        P.prism_block_select(self.p, self.nblk, self.qbar, self.kbar, self.row_ptr, self.col, self.nnz,
+                             self.ws_sel)
+
+    def attend(self):
+        P.prism_bsa_fwd(self.p, self.blocks, self.zone_blk_base, self.nblk, self.qp, self.kp, self.vp,
+                        self.row_ptr, self.col, self.op, self.lse)
+
+    def forward(self, q, k, v, audio=None, out=None):
+        """Natural-layout output O [N, heads, head_dim] bf16."""
+        self.indicator(v, audio)
+        self.assign()
+        self.permute(q, k, v)
+        self.select()
+        self.attend()
+        if out is None:
+            out = torch.empty(self.N, self.heads, self.D, dtype=torch.bfloat16, device=self.device)
+        P.prism_unpermute(self.p, self.shape_id, self.op, out)
+        return out
+
+    # -- backward -----------------------------------------------------------
+    def _bwd_buffers(self):
+        if self._bwd is None:
+            ws, _ = P.prism_workspace_size(self.p, P.PRISM_WS_BWD, self.col.numel())
+            self._bwd = dict(
+                dop=torch.empty_like(self.qp), dqp=torch.empty_like(self.qp), dkp=torch.empty_like(self.qp),
+                dvp=torch.empty_like(self.qp), ws=torch.empty(ws, dtype=torch.uint8, device=self.device))
+        return self._bwd
+
+    def attend_backward(self):
+        b = self._bwd_buffers()
+        P.prism_bsa_bwd(self.p, self.blocks, self.zone_blk_base, self.nblk, self.qp, self.kp, self.vp, self.op,
+                        b["dop"], self.lse, self.row_ptr, self.col, self.nnz, b["dqp"], b["dkp"], b["dvp"],
+                        b["ws"])
+
+    def backward(self, dout, dq=None, dk=None, dv=None):
+        """Gradients (dQ, dK, dV) in natural layout for the last forward's selection."""
+        b = self._bwd_buffers()
+        P.prism_permute(self.p, self.shape_id, self.zone_blk_base, dout, b["dop"], None)
+        self.attend_backward()
+        outs = []
+        for src, dst in ((b["dqp"], dq), (b["dkp"], dk), (b["dvp"], dv)):
+            if dst is None:
+                dst = torch.empty(self.N, self.heads, self.D, dtype=torch.bfloat16, device=self.device)
+            P.prism_unpermute(self.p, self.shape_id, src, dst)
+            outs.append(dst)
+        return tuple(outs)
+
+    # -- host views (for tests and reports) ---------------------------------
+    def host_layout(self):
+        nb = int(self.nblk.item())
+        return dict(nblk=nb, shape_id=self.shape_id.cpu().numpy(), zone_blk_base=self.zone_blk_base.cpu().numpy(),
+                    blocks=self.blocks[:nb].cpu().numpy())
+
+    def host_csr(self):
+        """Per-head CSR (row_ptr [heads, nblk+1] relative to each head, cols list)."""
+        nb = int(self.nblk.item())
+        rp = self.row_ptr.cpu().numpy().astype("int64")
+        col = self.col.cpu().numpy()
+        out_rp, out_cols = [], []
+        for h in range(self.heads):
+            r = rp[h * self.cap: h * self.cap + nb + 1]
+            out_rp.append(r - r[0])
+            out_cols.append(col[r[0]:r[-1]].astype("int64"))
+        import numpy as np
+        return np.stack(out_rp), out_cols

@@ -1,0 +1,412 @@
+// C ABI of the Prism sparse-attention library (declared in include/prism.h).
+// The whole library is this one translation unit: it includes the kernel
+// headers, validates arguments on the host, lays out workspaces and launches.
+#include <cmath>
+#include <cstdio>
+#include <string>
+
+#include "attn_mma_bwd.cuh"
+#include "indicator.cuh"
+#include "permute.cuh"
+#include "select.cuh"
+
+namespace prism {
+
+static thread_local std::string t_error;
+
+int fail(int code, const char *msg) {
+  t_error = msg ? msg : "";
+  return code;
+}
+
+struct Dims {
+  int T, H, W, heads, D, ZT, ZY, ZX;
+  int64_t N, Z, cap, C;
+};
+
+static int check_params(const prism_params *p, Dims *d) {
+  if (!p) return fail(PRISM_EINVAL, "params is NULL");
+  if (p->T <= 0 || p->H <= 0 || p->W <= 0 || p->T % kZone || p->H % kZone || p->W % kZone)
+    return fail(PRISM_EINVAL, "token grid T, H, W must be positive multiples of 8");
+  if (p->heads <= 0) return fail(PRISM_EINVAL, "heads must be positive");
+  if (p->head_dim != 64 && p->head_dim != 128) return fail(PRISM_EINVAL, "head_dim must be 64 or 128");
+  d->T = p->T; d->H = p->H; d->W = p->W; d->heads = p->heads; d->D = p->head_dim;
+  d->ZT = p->T / kZone; d->ZY = p->H / kZone; d->ZX = p->W / kZone;
+  d->N = (int64_t)p->T * p->H * p->W;
+  d->Z = d->N / kZoneTokens;
+  d->cap = d->Z * kMaxBlocksPerZone;
+  d->C = (int64_t)p->heads * p->head_dim;
+  if (d->Z > 65535) return fail(PRISM_EINVAL, "grid has more than 65535 macro-zones");
+  return PRISM_OK;
+}
+
+static bool aligned16(const void *ptr) { return ((uintptr_t)ptr & 15u) == 0; }
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+static cudaStream_t as_stream(prism_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+static float eff_scale(const prism_params *p) {
+  return p->scale > 0.f ? p->scale : 1.f / std::sqrt((float)p->head_dim);
+}
+
+// Workspace layouts.
+struct IndicatorWs {
+  size_t part, rec, total;
+  int nslab;
+  IndicatorWs(const Dims &d) {
+    nslab = (int)((d.C + kSlab - 1) / kSlab);
+    part = 0;
+    rec = align256((size_t)d.Z * nslab * 3 * sizeof(float));
+    total = rec + align256((size_t)d.Z * kZoneRec * sizeof(double));
+  }
+};
+struct SelectWs {
+  size_t cnt, key, q, part, scores, fixed, per_head;
+  int64_t R, nchunk;
+  SelectWs(const Dims &d) {
+    R = (int64_t)d.heads * d.cap;
+    nchunk = (R + kScanChunk - 1) / kScanChunk;
+    cnt = 0;
+    key = cnt + align256(R * 4);
+    q = key + align256(R * 4);
+    part = q + align256(R * 4);
+    scores = part + align256(nchunk * 8);
+    fixed = scores;
+    per_head = align256((size_t)d.cap * d.cap * sizeof(float));
+  }
+};
+struct BwdWs {
+  size_t delta, ccnt, col_ptr, fill, part, tot, row_idx, total;
+  int64_t R, nchunk;
+  BwdWs(const Dims &d, int64_t col_capacity) {
+    R = (int64_t)d.heads * d.cap;
+    nchunk = (R + kScanChunk - 1) / kScanChunk;
+    delta = 0;
+    ccnt = align256((size_t)d.heads * d.N * 4);
+    col_ptr = ccnt + align256(R * 4);
+    fill = col_ptr + align256((R + 1) * 4);
+    part = fill + align256(R * 4);
+    tot = part + align256(nchunk * 8);
+    row_idx = tot + 256;
+    total = row_idx + align256((size_t)(col_capacity > 0 ? col_capacity : 0) * 4);
+  }
+};
+
+static int launch_scan(const int32_t *cnt, int64_t R, long long *part, int64_t nchunk, int64_t capacity,
+                       int32_t *row_ptr, int64_t *nnz, cudaStream_t st) {
+  scan_partial_kernel<<<(unsigned)nchunk, kScanThreads, 0, st>>>(cnt, R, part);
+  scan_top_kernel<<<1, kScanThreads, 0, st>>>(part, (int)nchunk, capacity, nnz);
+  scan_final_kernel<<<(unsigned)nchunk, kScanThreads, 0, st>>>(cnt, R, part, nnz, capacity, row_ptr);
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+}  // namespace prism
+
+using namespace prism;
+
+extern "C" {
+
+const char *prism_last_error(void) { return t_error.c_str(); }
+
+int prism_device_status(prism_stream stream) {
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return fail(PRISM_ECUDA, cudaGetErrorString(e));
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int));
+  if (e != cudaSuccess) return fail(PRISM_ECUDA, cudaGetErrorString(e));
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return fail(PRISM_ECUDA, cudaGetErrorString(e));
+    const char *what = v == PRISM_ECAPACITY ? "selected pairs exceed col_capacity"
+                       : v == PRISM_ETIMEOUT ? "a bounded device wait timed out"
+                                             : "a device index check failed";
+    return fail(v, what);
+  }
+  return PRISM_OK;
+}
+
+int prism_workspace_size(const prism_params *p, int kind, int64_t col_capacity, size_t *bytes,
+                         size_t *bytes_all_heads) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!bytes) return fail(PRISM_EINVAL, "bytes is NULL");
+  size_t all = 0;
+  switch (kind) {
+    case PRISM_WS_INDICATOR: *bytes = all = IndicatorWs(d).total; break;
+    case PRISM_WS_SELECT: {
+      SelectWs w(d);
+      *bytes = w.fixed + w.per_head;
+      all = w.fixed + w.per_head * d.heads;
+      break;
+    }
+    case PRISM_WS_FWD: *bytes = all = 0; break;
+    case PRISM_WS_BWD: *bytes = all = BwdWs(d, col_capacity).total; break;
+    default: return fail(PRISM_EINVAL, "unknown workspace kind");
+  }
+  if (bytes_all_heads) *bytes_all_heads = all;
+  return PRISM_OK;
+}
+
+int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, const float *audio, float *g,
+                         float *rho, float *debug, void *workspace, size_t ws_bytes, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!V || !g || !rho) return fail(PRISM_EINVAL, "V, g and rho must be non-NULL");
+  if (!aligned16(V)) return fail(PRISM_EINVAL, "V must be 16-byte aligned");
+  if (v_dtype != PRISM_BF16 && v_dtype != PRISM_F32) return fail(PRISM_EINVAL, "V dtype must be bf16 or f32");
+  IndicatorWs w(d);
+  if (!workspace || ws_bytes < w.total) return fail(PRISM_EINVAL, "indicator workspace too small");
+  cudaStream_t st = as_stream(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *part = reinterpret_cast<float *>(ws + w.part);
+  double *rec = reinterpret_cast<double *>(ws + w.rec);
+  dim3 grid(w.nslab, (unsigned)d.Z);
+  if (v_dtype == PRISM_BF16)
+    zone_stats_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(V), (int)d.C,
+                                                            d.H, d.W, d.ZY, d.ZX, part);
+  else
+    zone_stats_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(V), (int)d.C, d.H, d.W, d.ZY,
+                                                    d.ZX, part);
+  zone_finish_kernel<<<(unsigned)d.Z, 64, 0, st>>>(part, w.nslab, (int)d.C, audio, d.H, d.W, d.ZY, d.ZX, rec);
+  zone_final_kernel<<<1, 1024, 0, st>>>(rec, (int)d.Z, audio != nullptr, p->eps, g, rho, debug);
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+int prism_assign_blocks(const prism_params *p, const float *g, const float *rho, uint8_t *shape_id,
+                        int32_t *zone_blk_base, prism_block *blocks, int32_t *nblk, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!g || !rho || !shape_id || !zone_blk_base || !blocks || !nblk)
+    return fail(PRISM_EINVAL, "assign_blocks: NULL argument");
+  assign_blocks_kernel<<<1, 1024, 0, as_stream(stream)>>>(g, rho, (int)d.Z, p->tau128, p->tau256, shape_id,
+                                                          zone_blk_base, blocks, nblk);
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+int prism_permute(const prism_params *p, const uint8_t *shape_id, const int32_t *zone_blk_base, const void *x,
+                  int x_dtype, void *x_perm, float *pooled, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!shape_id || !x || !x_perm || (pooled && !zone_blk_base)) return fail(PRISM_EINVAL, "permute: NULL argument");
+  if (!aligned16(x) || !aligned16(x_perm)) return fail(PRISM_EINVAL, "permute: tensors must be 16-byte aligned");
+  if (x_dtype != PRISM_BF16 && x_dtype != PRISM_F32) return fail(PRISM_EINVAL, "permute: dtype must be bf16 or f32");
+  cudaStream_t st = as_stream(stream);
+  dim3 grid(d.heads, (unsigned)d.Z);
+  auto *xp = static_cast<__nv_bfloat16 *>(x_perm);
+#define PRISM_PERMUTE(TIN, DD)                                                                                \
+  permute_kernel<TIN, DD><<<grid, 256, 0, st>>>(static_cast<const TIN *>(x), d.heads, d.N, d.H, d.W, d.ZY, d.ZX, \
+                                                shape_id, zone_blk_base, d.cap, xp, pooled)
+  if (x_dtype == PRISM_BF16) {
+    if (d.D == 128) PRISM_PERMUTE(__nv_bfloat16, 128); else PRISM_PERMUTE(__nv_bfloat16, 64);
+  } else {
+    if (d.D == 128) PRISM_PERMUTE(float, 128); else PRISM_PERMUTE(float, 64);
+  }
+#undef PRISM_PERMUTE
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+int prism_unpermute(const prism_params *p, const uint8_t *shape_id, const void *x_perm, int in_dtype, void *x,
+                    int out_dtype, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!shape_id || !x || !x_perm) return fail(PRISM_EINVAL, "unpermute: NULL argument");
+  if (!aligned16(x) || !aligned16(x_perm)) return fail(PRISM_EINVAL, "unpermute: tensors must be 16-byte aligned");
+  if ((in_dtype != PRISM_BF16 && in_dtype != PRISM_F32) || (out_dtype != PRISM_BF16 && out_dtype != PRISM_F32))
+    return fail(PRISM_EINVAL, "unpermute: dtype must be bf16 or f32");
+  cudaStream_t st = as_stream(stream);
+  dim3 grid(d.heads, (unsigned)d.Z);
+#define PRISM_UNPERMUTE(TIN, TOUT, DD)                                                                        \
+  unpermute_kernel<TIN, TOUT, DD><<<grid, 256, 0, st>>>(static_cast<const TIN *>(x_perm), d.heads, d.N, d.H, \
+                                                        d.W, d.ZY, d.ZX, shape_id, static_cast<TOUT *>(x))
+#define PRISM_UNPERMUTE_D(TIN, TOUT) \
+  do { if (d.D == 128) PRISM_UNPERMUTE(TIN, TOUT, 128); else PRISM_UNPERMUTE(TIN, TOUT, 64); } while (0)
+  if (in_dtype == PRISM_BF16 && out_dtype == PRISM_BF16) PRISM_UNPERMUTE_D(__nv_bfloat16, __nv_bfloat16);
+  else if (in_dtype == PRISM_BF16) PRISM_UNPERMUTE_D(__nv_bfloat16, float);
+  else if (out_dtype == PRISM_BF16) PRISM_UNPERMUTE_D(float, __nv_bfloat16);
+  else PRISM_UNPERMUTE_D(float, float);
+#undef PRISM_UNPERMUTE_D
+#undef PRISM_UNPERMUTE
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+int prism_block_select(const prism_params *p, const int32_t *nblk, const float *q_pooled, const float *k_pooled,
+                       int32_t *row_ptr, int32_t *col, int64_t col_capacity, int64_t *nnz, void *workspace,
+                       size_t ws_bytes, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!nblk || !q_pooled || !k_pooled || !row_ptr || !nnz || (!col && col_capacity > 0))
+    return fail(PRISM_EINVAL, "block_select: NULL argument");
+  if (!aligned16(q_pooled) || !aligned16(k_pooled)) return fail(PRISM_EINVAL, "block_select: pooled must be 16-byte aligned");
+  if (p->top_k < 1) return fail(PRISM_EINVAL, "top_k must be >= 1");
+  if (!(p->top_p > 0.f && p->top_p <= 1.f)) return fail(PRISM_EINVAL, "top_p must be in (0, 1]");
+  const size_t key_bytes = (size_t)d.cap * 4;
+  if (key_bytes + sizeof(SelShared) > 227 * 1024) return fail(PRISM_EINVAL, "too many blocks per head for selection");
+  SelectWs w(d);
+  if (!workspace || ws_bytes < w.fixed + w.per_head) return fail(PRISM_EINVAL, "select workspace too small");
+  const int hp = (int)std::min<int64_t>(d.heads, (int64_t)((ws_bytes - w.fixed) / w.per_head));
+  const bool once = hp >= d.heads;
+  cudaStream_t st = as_stream(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  int32_t *cnt = reinterpret_cast<int32_t *>(ws + w.cnt);
+  uint32_t *ckey = reinterpret_cast<uint32_t *>(ws + w.key);
+  int32_t *cq = reinterpret_cast<int32_t *>(ws + w.q);
+  long long *part = reinterpret_cast<long long *>(ws + w.part);
+  float *S = reinterpret_cast<float *>(ws + w.scores);
+  const float scale = eff_scale(p);
+  const unsigned tiles = (unsigned)((d.cap + 63) / 64);
+  cudaFuncSetAttribute(row_cut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)key_bytes);
+  for (int h0 = 0; h0 < d.heads; h0 += hp) {
+    const int nh = std::min(hp, d.heads - h0);
+    block_scores_kernel<<<dim3(tiles, tiles, nh), 256, 0, st>>>(q_pooled, k_pooled, d.D, d.cap, nblk, h0, scale, S);
+    row_cut_kernel<<<dim3((unsigned)d.cap, nh), kSelThreads, key_bytes, st>>>(S, d.cap, nblk, h0, p->top_k,
+                                                                               p->top_p, cnt, ckey, cq);
+  }
+  PRISM_CUDA_CHECK_LAUNCH();
+  rc = launch_scan(cnt, w.R, part, w.nchunk, col_capacity, row_ptr, nnz, st);
+  if (rc) return rc;
+  for (int h0 = 0; h0 < d.heads; h0 += hp) {
+    const int nh = std::min(hp, d.heads - h0);
+    if (!once)
+      block_scores_kernel<<<dim3(tiles, tiles, nh), 256, 0, st>>>(q_pooled, k_pooled, d.D, d.cap, nblk, h0, scale, S);
+    emit_kernel<<<dim3((unsigned)d.cap, nh), kSelThreads, 0, st>>>(S, d.cap, nblk, h0, ckey, cq, row_ptr, nnz,
+                                                                  col_capacity, col);
+  }
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+}  // extern "C"
+
+static int check_attn(const prism_params *p, Dims *d, const void *blocks, const void *zbb, const void *nblk,
+                      const void *const *tensors, int nt, const void *row_ptr, const void *col) {
+  int rc = check_params(p, d);
+  if (rc) return rc;
+  if (!blocks || !zbb || !nblk || !row_ptr || !col) return fail(PRISM_EINVAL, "attention: NULL argument");
+  for (int t = 0; t < nt; ++t) {
+    if (!tensors[t]) return fail(PRISM_EINVAL, "attention: NULL tensor");
+    if (!aligned16(tensors[t])) return fail(PRISM_EINVAL, "attention: tensors must be 16-byte aligned");
+  }
+  if (d->N / 64 > 0x7fffffffLL || d->heads > 65535) return fail(PRISM_EINVAL, "attention: grid too large");
+  return PRISM_OK;
+}
+
+extern "C" {
+
+int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
+                  const int32_t *nblk, const void *q, const void *k, const void *v, const int32_t *row_ptr,
+                  const int32_t *col, void *o, float *lse, void *workspace, size_t ws_bytes,
+                  prism_stream stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  Dims d;
+  const void *tens[5] = {q, k, v, o, lse};
+  int rc = check_attn(p, &d, blocks, zone_blk_base, nblk, tens, 5, row_ptr, col);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  const float scale_log2 = eff_scale(p) * kLog2e;
+  dim3 grid((unsigned)(d.N / 64), d.heads);
+  auto Q = static_cast<const __nv_bfloat16 *>(q), K = static_cast<const __nv_bfloat16 *>(k),
+       Vv = static_cast<const __nv_bfloat16 *>(v);
+  auto O = static_cast<__nv_bfloat16 *>(o);
+  if (d.D == 128) {
+    const int smem = 5 * 64 * 128 * 2;
+    cudaFuncSetAttribute(bsa_fwd_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    bsa_fwd_mma_kernel<128><<<grid, 128, smem, st>>>(Q, K, Vv, blocks, zone_blk_base, row_ptr, col, d.N, d.cap,
+                                                     scale_log2, O, lse);
+  } else {
+    const int smem = 5 * 64 * 64 * 2;
+    bsa_fwd_mma_kernel<64><<<grid, 128, smem, st>>>(Q, K, Vv, blocks, zone_blk_base, row_ptr, col, d.N, d.cap,
+                                                    scale_log2, O, lse);
+  }
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+}  // extern "C"
+
+template <int D>
+static void launch_bwd_attn(const Dims &d, dim3 grid, cudaStream_t st, const __nv_bfloat16 *Q,
+                            const __nv_bfloat16 *K, const __nv_bfloat16 *Vv, const __nv_bfloat16 *dO,
+                            const float *lse, const float *delta, const prism_block *blocks,
+                            const int32_t *zbb, const int32_t *row_ptr, const int32_t *col,
+                            const int32_t *col_ptr, const int32_t *row_idx, float scale, __nv_bfloat16 *dq,
+                            __nv_bfloat16 *dk, __nv_bfloat16 *dv) {
+  const int smem_kv = 6 * 64 * D * 2 + 2 * 2 * 64 * 4;
+  const int smem_q = 6 * 64 * D * 2;
+  cudaFuncSetAttribute(bsa_dkdv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
+  cudaFuncSetAttribute(bsa_dq_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
+  bsa_dkdv_mma_kernel<D><<<grid, 128, smem_kv, st>>>(Q, K, Vv, dO, lse, delta, blocks, zbb, col_ptr, row_idx,
+                                                      d.N, d.cap, scale, dk, dv);
+  bsa_dq_mma_kernel<D><<<grid, 128, smem_q, st>>>(Q, K, Vv, dO, lse, delta, blocks, zbb, row_ptr, col, d.N,
+                                                   d.cap, scale, dq);
+}
+
+extern "C" {
+
+int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
+                  const int32_t *nblk, const void *q, const void *k, const void *v, const void *o,
+                  const void *dout, const float *lse, const int32_t *row_ptr, const int32_t *col,
+                  const int64_t *nnz, int64_t col_capacity, void *dq, void *dk, void *dv, void *workspace,
+                  size_t ws_bytes, prism_stream stream) {
+  Dims d;
+  const void *tens[10] = {q, k, v, o, dout, lse, dq, dk, dv, workspace};
+  int rc = check_attn(p, &d, blocks, zone_blk_base, nblk, tens, 10, row_ptr, col);
+  if (rc) return rc;
+  if (!nnz) return fail(PRISM_EINVAL, "bwd: nnz is NULL");
+  BwdWs w(d, col_capacity);
+  if (ws_bytes < w.total) return fail(PRISM_EINVAL, "bwd workspace too small");
+  const int64_t sort_bytes = [&] { int64_t p2 = 1; while (p2 < d.cap) p2 <<= 1; return p2 * 4; }();
+  if (sort_bytes > 227 * 1024) return fail(PRISM_EINVAL, "too many blocks per head for the backward");
+  cudaStream_t st = as_stream(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  float *delta = reinterpret_cast<float *>(ws + w.delta);
+  int32_t *ccnt = reinterpret_cast<int32_t *>(ws + w.ccnt);
+  int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + w.col_ptr);
+  int32_t *fill = reinterpret_cast<int32_t *>(ws + w.fill);
+  long long *part = reinterpret_cast<long long *>(ws + w.part);
+  int32_t *row_idx = reinterpret_cast<int32_t *>(ws + w.row_idx);
+  auto O = static_cast<const __nv_bfloat16 *>(o), dO = static_cast<const __nv_bfloat16 *>(dout);
+  const int64_t rows = (int64_t)d.heads * d.N;
+  if (d.D == 128)
+    bwd_delta_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, dO, rows, delta);
+  else
+    bwd_delta_kernel<64><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, dO, rows, delta);
+  cudaMemsetAsync(ccnt, 0, w.R * 4, st);
+  cudaMemsetAsync(fill, 0, w.R * 4, st);
+  dim3 rgrid((unsigned)d.cap, d.heads);
+  csc_count_kernel<<<rgrid, 256, 0, st>>>(row_ptr, col, d.cap, nblk, ccnt);
+  // column counts -> column pointers (their total equals the selection's nnz)
+  int64_t *tot = reinterpret_cast<int64_t *>(ws + w.tot);
+  rc = launch_scan(ccnt, w.R, part, w.nchunk, col_capacity, col_ptr, tot, st);
+  if (rc) return rc;
+  csc_fill_kernel<<<rgrid, 256, 0, st>>>(row_ptr, col, d.cap, nblk, col_ptr, fill, row_idx);
+  cudaFuncSetAttribute(csc_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sort_bytes);
+  csc_sort_kernel<<<rgrid, 512, sort_bytes, st>>>(col_ptr, d.cap, nblk, row_idx);
+  PRISM_CUDA_CHECK_LAUNCH();
+  dim3 grid((unsigned)(d.N / 64), d.heads);
+  auto Q = static_cast<const __nv_bfloat16 *>(q), K = static_cast<const __nv_bfloat16 *>(k),
+       Vv = static_cast<const __nv_bfloat16 *>(v);
+  const float scale = eff_scale(p);
+  if (d.D == 128)
+    launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
+                         row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
+                         static_cast<__nv_bfloat16 *>(dv));
+  else
+    launch_bwd_attn<64>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
+                        row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
+                        static_cast<__nv_bfloat16 *>(dv));
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,217 @@
+/*
+ * prism.h -- C ABI of the B200 (sm_100a) implementation of Prism's dynamic
+ * block-sparse video self-attention ("Prism: Dynamic Sparse Attention for
+ * Native 2K Joint Video-Audio Generation Model Training", arXiv 2610.05416).
+ *
+ * The path, in call order (forward):
+ *   prism_zone_indicator -> prism_assign_blocks -> prism_permute (Q, K, V)
+ *   -> prism_block_select -> prism_bsa_fwd -> prism_unpermute (O)
+ * and backward:
+ *   prism_permute (dO) -> prism_bsa_bwd -> prism_unpermute (dQ, dK, dV)
+ *
+ * Conventions shared by every entry point
+ *   - All pointers are DEVICE pointers unless a comment says otherwise; the
+ *     caller owns every buffer.  No entry point allocates device memory:
+ *     scratch comes in through (workspace, ws_bytes), sized by
+ *     prism_workspace_size().
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  Counts produced on the device (the number of
+ *     blocks, the number of selected pairs) stay on the device; buffers are
+ *     sized by the upper bounds stated below so that no call needs a host sync.
+ *   - Return value: PRISM_OK, or a negative status for errors found on the
+ *     host before launch (PRISM_EINVAL, PRISM_ECUDA).  Errors found by a
+ *     kernel (capacity overflow, a bounded wait that timed out, an index out of
+ *     range) are latched in a device status word that prism_device_status()
+ *     returns and clears.  prism_last_error() gives a message for the last
+ *     non-zero status of the calling thread.  Nothing traps or aborts.
+ *   - Layouts.  Natural token order n = (t*H + y)*W + x.  "Natural" tensors
+ *     are [N, heads, head_dim]; "permuted" tensors are [heads, N, head_dim]
+ *     with the tokens in zone-local block order (see prism_permute), so every
+ *     block of every head is one contiguous [B, head_dim] tile.
+ *   - Sizes.  Z = N/512 zones; a zone holds 512/B blocks with B in
+ *     {64,128,256}, so the block count nblk <= NBLK_CAP = 8*Z.  Per-head block
+ *     arrays are strided by NBLK_CAP.
+ */
+#ifndef PRISM_H
+#define PRISM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define PRISM_OK 0
+#define PRISM_EINVAL (-1)    /* bad argument: null, misaligned, unsupported size */
+#define PRISM_ECAPACITY (-2) /* selected pairs exceed col_capacity (device-reported) */
+#define PRISM_ECUDA (-3)     /* a CUDA runtime call failed */
+#define PRISM_ETIMEOUT (-4)  /* a bounded device wait gave up (device-reported) */
+#define PRISM_EBOUNDS (-5)   /* a device index check failed (device-reported) */
+
+/* element types */
+#define PRISM_BF16 0
+#define PRISM_F32 1
+
+/* workspace kinds for prism_workspace_size */
+#define PRISM_WS_INDICATOR 0
+#define PRISM_WS_SELECT 1
+#define PRISM_WS_FWD 2
+#define PRISM_WS_BWD 3
+
+typedef void *prism_stream; /* cudaStream_t */
+
+/*
+ * Problem statement (Method, and the knobs of the selection):
+ *   T, H, W   token grid; each a positive multiple of the 8x8x8 macro-zone
+ *             (Key ideas, "Macro-Zone Partitioning").
+ *   heads, head_dim   attention heads and per-head width; head_dim 64 or 128.
+ *   tau128, tau256    density thresholds of Method §2 (0.5 and 0.25).
+ *   eps       the epsilon of the composite indicator g_d (Method §1); 1e-4.
+ *   top_k     minimum number of key blocks per query block (Method §3), >= 1.
+ *   top_p     cumulative probability mass to keep (Method §3), in (0, 1].
+ *   scale     softmax scale for block scores and attention; 0 means
+ *             1/sqrt(head_dim).
+ */
+typedef struct {
+  int32_t T, H, W;
+  int32_t heads, head_dim;
+  float tau128, tau256;
+  float eps;
+  int32_t top_k;
+  float top_p;
+  float scale;
+} prism_params;
+
+/* One block of the zone-local layout: permuted rows [start, start+size) of
+ * every head, inside zone `zone`, of canonical shape index `shape`. */
+typedef struct {
+  int32_t start, size, zone, shape;
+} prism_block;
+
+/* Bytes of workspace an entry point needs (kind = PRISM_WS_*).  For
+ * PRISM_WS_SELECT the amount is the minimum (one head of block scores at a
+ * time); more lets more heads run per pass, up to `*bytes_all_heads`.
+ * col_capacity matters for PRISM_WS_BWD only.  Host-only; returns a status. */
+int prism_workspace_size(const prism_params *p, int kind, int64_t col_capacity,
+                         size_t *bytes, size_t *bytes_all_heads);
+
+/*
+ * Method §1 and the density of §2: per macro-zone m, the directional video
+ * variances sigma^2_{v,d}(m) of the mean-pooled V along T, H and W (averaged
+ * over all heads*head_dim channels), r_{v,d} = sigma^2_{v,d}/sum, the audio
+ * coupling abar(m) = zone mean of a / global max of a, the normalised audio
+ * directional variance vhat_{a,d} (a pooled like V), the composite indicator
+ * g_d = r_{v,d} + abar*vhat_{a,d} + eps and the density
+ * rho(m) = (info(m)/max info + abar(m))/2 with info = sum_d sigma^2_{v,d}.
+ *   V      natural [N, heads, head_dim], dtype PRISM_BF16 or PRISM_F32,
+ *          16-byte aligned.
+ *   audio  [N] float, nullable: NULL (first layer, no cached norms) means
+ *          abar = vhat = 0.
+ *   g      out [Z, 3] float (T, H, W);  rho  out [Z] float.
+ *   debug  out, nullable: [Z, 8] float = sigma2_v[3], info, abar, vhat_a[3].
+ *   workspace  >= prism_workspace_size(PRISM_WS_INDICATOR) bytes.
+ */
+int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, const float *audio,
+                         float *g, float *rho, float *debug, void *workspace, size_t ws_bytes,
+                         prism_stream stream);
+
+/*
+ * Method §2: block volume B(m) (rho >= tau128 -> 64, tau256 <= rho < tau128 ->
+ * 128, else 256), optimal log2 edges l*_d = -1/2 log2 g_d + 1/3(S + 1/2 sum
+ * log2 g), and the nearest of the 16 candidate shapes (edges in {2,4,8},
+ * product B; canonical order volume then (bT,bH,bW) ascending; distance ties
+ * within 1e-9 go to the lowest index).  Decisions are taken in double.
+ *   g [Z,3], rho [Z]        in (as produced by prism_zone_indicator)
+ *   shape_id [Z]            out, canonical shape index
+ *   zone_blk_base [Z+1]     out, first block of each zone (exclusive scan)
+ *   blocks [8Z]             out, block table in zone-local order
+ *   nblk [1]                out, number of blocks
+ */
+int prism_assign_blocks(const prism_params *p, const float *g, const float *rho, uint8_t *shape_id,
+                        int32_t *zone_blk_base, prism_block *blocks, int32_t *nblk,
+                        prism_stream stream);
+
+/*
+ * Zone-local token permutation with fused block mean-pooling (Method §3's
+ * block representatives).  Zone m owns permuted rows [512m, 512m+512); inside
+ * it the blocks follow raster order over the (8/bT, 8/bH, 8/bW) block grid and
+ * the tokens of a block follow raster (t, y, x).
+ *   x        natural [N, heads, head_dim], PRISM_BF16 or PRISM_F32, 16-B aligned
+ *   x_perm   out, permuted [heads, N, head_dim] bf16
+ *   pooled   out, nullable: [heads, 8Z, head_dim] float, mean of each block's
+ *            rows (computed from x in its own precision)
+ */
+int prism_permute(const prism_params *p, const uint8_t *shape_id, const int32_t *zone_blk_base,
+                  const void *x, int x_dtype, void *x_perm, float *pooled, prism_stream stream);
+
+/* Inverse of prism_permute: permuted [heads, N, head_dim] (in_dtype) ->
+ * natural [N, heads, head_dim] (out_dtype). */
+int prism_unpermute(const prism_params *p, const uint8_t *shape_id, const void *x_perm,
+                    int in_dtype, void *x, int out_dtype, prism_stream stream);
+
+/*
+ * Method §3: block scores s_ij = scale * Qbar_i . Kbar_j (float), block
+ * probabilities P_i = softmax_j over the head's blocks, and the hybrid set
+ * S_i = Top-k(P_i, k) U Top-p(P_i, p): key blocks ranked by (score
+ * descending, index ascending); S_i is the longest of the first min(k, nblk)
+ * and the shortest prefix whose mass reaches p (mass summed in 2^-40 fixed
+ * point).  Output is a CSR per head over rows h*8Z + i, columns ascending.
+ *   nblk [1]              in (device), from prism_assign_blocks
+ *   q_pooled, k_pooled    in [heads, 8Z, head_dim] float
+ *   row_ptr               out [heads*8Z + 1] int32 (rows i >= nblk are empty)
+ *   col                   out [col_capacity] int32
+ *   nnz [1]               out (device) int64, total selected pairs.  If it
+ *                         exceeds col_capacity nothing is written to col and
+ *                         the device status becomes PRISM_ECAPACITY.
+ *   workspace             >= the PRISM_WS_SELECT minimum
+ */
+int prism_block_select(const prism_params *p, const int32_t *nblk, const float *q_pooled,
+                       const float *k_pooled, int32_t *row_ptr, int32_t *col, int64_t col_capacity,
+                       int64_t *nnz, void *workspace, size_t ws_bytes, prism_stream stream);
+
+/*
+ * Method §3: block-sparse attention forward, online softmax, bidirectional:
+ * for each query row r of block i, O_r = softmax(scale q_r K^T) V over the
+ * tokens of the key blocks in S_i; LSE_r = natural log of the softmax
+ * denominator (including the max).
+ *   blocks, nblk          from prism_assign_blocks; zone_blk_base likewise
+ *   q, k, v               permuted [heads, N, head_dim] bf16, 16-B aligned
+ *   row_ptr, col          CSR from prism_block_select
+ *   o                     out permuted [heads, N, head_dim] bf16
+ *   lse                   out [heads, N] float
+ */
+int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
+                  const int32_t *nblk, const void *q, const void *k, const void *v,
+                  const int32_t *row_ptr, const int32_t *col, void *o, float *lse, void *workspace,
+                  size_t ws_bytes, prism_stream stream);
+
+/*
+ * Backward of prism_bsa_fwd for the fixed selection: with P the attention
+ * probabilities, dV = P^T dO, dP = dO V^T, D_r = rowsum(dO o O),
+ * dS = P (dP - D), dQ = scale dS K, dK = scale dS^T Q.
+ *   o, dout               permuted [heads, N, head_dim] bf16 (forward output, its gradient)
+ *   lse                   [heads, N] float from prism_bsa_fwd
+ *   nnz, col_capacity     as returned to / given to prism_block_select
+ *   dq, dk, dv            out permuted [heads, N, head_dim] bf16
+ *   workspace             >= prism_workspace_size(PRISM_WS_BWD, col_capacity)
+ */
+int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
+                  const int32_t *nblk, const void *q, const void *k, const void *v, const void *o,
+                  const void *dout, const float *lse, const int32_t *row_ptr, const int32_t *col,
+                  const int64_t *nnz, int64_t col_capacity, void *dq, void *dk, void *dv,
+                  void *workspace, size_t ws_bytes, prism_stream stream);
+
+/* Synchronises `stream`, returns the latched device status (PRISM_OK or one
+ * of PRISM_ECAPACITY / PRISM_ETIMEOUT / PRISM_EBOUNDS) and clears it. */
+int prism_device_status(prism_stream stream);
+
+/* Message for the last non-zero status returned to the calling thread. */
+const char *prism_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PRISM_H */

@@ -1,0 +1,90 @@
+"""Shared test utilities: comparisons, CSR conversion, near-tie analysis."""
+
+import math
+
+import numpy as np
+import torch
+
+# Attention tolerance (bf16 storage, fp32 accumulation) against fp64.
+REL_RMS_TOL = 1e-2
+MAX_ABS_TOL = 3e-2
+
+
+def f64(t):
+    """Exact float64 copy of a (CPU or GPU) tensor."""
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def rel_rms(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    return float(np.sqrt(np.mean((a - b) ** 2)) / max(np.sqrt(np.mean(b ** 2)), 1e-30))
+
+
+def assert_close_attn(got, ref, what):
+    rr = rel_rms(got, ref)
+    ma = float(np.max(np.abs(np.asarray(got, dtype=np.float64) - ref)))
+    assert rr <= REL_RMS_TOL and ma <= MAX_ABS_TOL, f"{what}: rel_rms={rr:.3e} max_abs={ma:.3e}"
+    return rr, ma
+
+
+def csr_to_device(row_ptr_h, cols_h, cap, device):
+    """Per-head CSR (oracle form) -> the library's global row_ptr [heads*cap+1] and col."""
+    heads, nb1 = row_ptr_h.shape
+    nb = nb1 - 1
+    rp = np.zeros(heads * cap + 1, dtype=np.int64)
+    cols = []
+    off = 0
+    for h in range(heads):
+        r = row_ptr_h[h]
+        rp[h * cap: h * cap + nb + 1] = off + r
+        rp[h * cap + nb + 1: (h + 1) * cap + 1] = off + r[-1]
+        off += int(r[-1])
+        cols.append(np.asarray(cols_h[h], dtype=np.int64))
+    col = np.concatenate(cols) if cols else np.zeros(0, dtype=np.int64)
+    return (torch.from_numpy(rp.astype(np.int32)).to(device),
+            torch.from_numpy(col.astype(np.int32)).to(device),
+            torch.tensor([off], dtype=torch.int64, device=device))
+
+
+def blocks_to_device(blocks, cap, device):
+    b = np.zeros((cap, 4), dtype=np.int32)
+    b[:len(blocks)] = blocks
+    return torch.from_numpy(b).to(device)
+
+
+def selection_row_ok(P_row, gpu_sel, ora_sel, top_k, top_p, score_tol=1e-4, mass_tol=1e-5):
+    """Exact match, or a valid alternative when the oracle's row is near a tie.
+
+    Returns (exact, valid).  A row is near a tie if two blocks straddling the
+    cut have probabilities within a relative score_tol, or the cumulative mass
+    at the cut is within mass_tol of p.  A valid alternative keeps every block
+    clearly above the cut, no block clearly below it, at least min(k, nblk)
+    blocks, and mass >= p - mass_tol.
+    """
+    gpu_sel = np.asarray(gpu_sel)
+    ora_sel = np.asarray(ora_sel)
+    if len(gpu_sel) == len(ora_sel) and np.array_equal(gpu_sel, ora_sel):
+        return True, True
+    n = len(P_row)
+    logp = np.log(np.maximum(P_row, 1e-300))
+    cut = len(ora_sel)
+    order = sorted(range(n), key=lambda j: (-P_row[j], j))
+    lo = logp[order[cut - 1]]
+    hi_thr = lo + score_tol * max(1.0, abs(lo))
+    lo_thr = lo - score_tol * max(1.0, abs(lo))
+    must = {j for j in range(n) if logp[j] > hi_thr}
+    never = {j for j in range(n) if logp[j] < lo_thr and j not in must}
+    gs = set(gpu_sel.tolist())
+    cum = P_row[gpu_sel].sum() if len(gpu_sel) else 0.0
+    valid = (must <= gs and not (gs & never) and len(gs) >= min(top_k, n)
+             and cum >= top_p - mass_tol and list(gpu_sel) == sorted(gs))
+    # also allow a boundary move of the top-p prefix by one element when the
+    # cumulative mass at the cut is within mass_tol of p
+    if not valid:
+        csum = np.cumsum(P_row[order])
+        near = abs(csum[cut - 1] - top_p) < mass_tol or (cut >= 2 and abs(csum[cut - 2] - top_p) < mass_tol)
+        if near and abs(len(gs) - cut) <= 1:
+            pref = set(order[:len(gs)])
+            valid = gs == pref
+    return False, valid

@@ -1,0 +1,69 @@
+"""The C ABI without a GPU: every symbol the header declares is exported, and
+host-side argument checks answer before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from dynamic_block_sparse_variance_b200 import build, prism as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared():
+    names = []
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"^(?:int|const char \*|size_t|void)\s*\*?\s*(prism_\w+)\(", text, re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return P.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(P.ENTRY_POINTS) <= set(names)
+
+
+def test_workspace_sizes(lib):
+    p = P.make_params(64, 96, 160, 24, 128, 32, 0.9)
+    ind, _ = P.prism_workspace_size(p, P.PRISM_WS_INDICATOR)
+    sel_min, sel_all = P.prism_workspace_size(p, P.PRISM_WS_SELECT)
+    bwd, _ = P.prism_workspace_size(p, P.PRISM_WS_BWD, 10**8)
+    cap = 8 * (64 * 96 * 160 // 512)
+    assert ind > 0 and sel_min >= cap * cap * 4 and sel_all >= 24 * cap * cap * 4
+    assert bwd >= 4 * 10**8
+
+
+@pytest.mark.parametrize("bad", [dict(T=7), dict(H=0), dict(head_dim=96), dict(heads=0)])
+def test_invalid_params_rejected_on_host(lib, bad):
+    kw = dict(T=8, H=16, W=16, heads=2, head_dim=64, top_k=2, top_p=0.9)
+    kw.update(bad)
+    p = P.make_params(**kw)
+    with pytest.raises(P.PrismError) as e:
+        P.prism_workspace_size(p, P.PRISM_WS_INDICATOR)
+    assert e.value.code == P.PRISM_EINVAL
+    rc = lib.prism_zone_indicator(ctypes.byref(p), None, 0, None, None, None, None, None, 0, None)
+    assert rc == P.PRISM_EINVAL
+    assert lib.prism_last_error()
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    p = P.make_params(8, 16, 16, 2, 64, 2, 0.9)
+    assert lib.prism_permute(ctypes.byref(p), None, None, None, 0, None, None, None) == P.PRISM_EINVAL
+    fake = ctypes.c_void_p(0x1001)
+    assert lib.prism_permute(ctypes.byref(p), fake, fake, fake, 0, fake, None, None) == P.PRISM_EINVAL
+    assert b"aligned" in lib.prism_last_error()
+    bad_p = P.make_params(8, 16, 16, 2, 64, 0, 0.9)
+    assert lib.prism_block_select(ctypes.byref(bad_p), fake, fake, fake, fake, fake, 0, fake, fake, 1 << 30,
+                                  None) == P.PRISM_EINVAL
