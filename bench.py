@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of the whole Prism sparse-attention step (forward + backward).
+
+One step = indicator -> block assignment -> permutation (Q, K, V) -> block
+selection -> sparse attention forward -> unpermute(O) -> permute(dO) ->
+sparse attention backward -> unpermute(dQ, dK, dV), on one synthetic batch
+already resident in HBM.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2k]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on a bounded sample
+
+Multi-GPU runs (torchrun) are independent replicas, one layer per GPU (weak
+scaling); there is no data-path collective.
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "block-sparse attn fwd+bwd ms & executed TFLOP/s (% bf16 peak) at 2K-like grid"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = dict(bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, hbm_gbs=6650.0)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="prism", choices=["prism", "reference"])
+    ap.add_argument("--workload", default="2k")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks --
+class ClockSampler:
+    """nvidia-smi samples of this GPU's SM clock and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.lines = []
+        try:
+            bus = torch.cuda.get_device_properties(device).pci_bus_id
+            self.target = ["-i", bus]
+        except Exception:
+            self.target = ["-i", str(torch.cuda.current_device())]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *self.target, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["nvidia-smi unavailable"])
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 8:
+                rows.append(parts)
+        if not rows:
+            return dict(sm_mhz=None, sm_max_mhz=None, reasons=["no samples"])
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[4 + k].lower().startswith("active")})
+        load = [s for s in sm if s > 0.5 * max(sm)] if sm else []
+        return dict(sm_mhz=statistics.median(load) if load else None, sm_max_mhz=max(mx) if mx else None,
+                    reasons=reasons, samples=len(rows))
+
+
+# ------------------------------------------------------------- counting --
+def executed_pairs(att):
+    """sum over heads, query blocks i and selected key blocks j of B_i * B_j."""
+    nb = int(att.nblk.item())
+    sizes = att.blocks[:nb, 1].to(torch.int64)
+    nnz = int(att.nnz.item())
+    total = 0
+    for h in range(att.heads):
+        rp = att.row_ptr[h * att.cap: h * att.cap + nb + 1].to(torch.int64)
+        cnt = rp[1:] - rp[:-1]
+        cols = att.col[int(rp[0]): int(rp[-1])].to(torch.int64)
+        rows = torch.repeat_interleave(torch.arange(nb, device=cols.device), cnt)
+        total += int((sizes[rows] * sizes[cols]).sum().item())
+    return total, nnz, nb, sizes
+
+
+# Algorithmic tensor-core FLOPs of each attention kernel, in units of
+# P = sum_h sum_i sum_{j in S_i} B_i B_j d: forward 4P (QK^T, PV); the key-side
+# backward kernel 8P (S, dP, dV, dK); the query-side one 2P (dQ; its S and dP
+# recomputation is extra work and not counted).
+KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_dkdv_mma_kernel": 8, "bsa_dq_mma_kernel": 2}
+
+
+# ------------------------------------------------------------ CPU oracle --
+def oracle_sample(inputs, wl, budget_s, seed=0, steps=1):
+    """Time the fp64 oracle on a bounded sample of the same workload.
+
+    The sample is the first 8-frame slab (one zone layer: 8 x H x W tokens,
+    all heads) of the benchmark's own inputs.  The indicator, block
+    assignment, permutation and pooling run in full on the slab; selection,
+    forward and backward run on query blocks drawn at random (seeded) until
+    the time budget is spent.  Returns executed attention TFLOP/s of the
+    sampled query blocks and the details.
+    """
+    from oracle import prism_oracle as po
+
+    plane = wl.H * wl.W
+    n_s = 8 * plane
+    f = lambda t: t[:n_s].detach().to("cpu", torch.float32).numpy()
+    q, k, v, do = (f(inputs[n]) for n in ("q", "k", "v", "dout"))
+    audio = None if inputs["audio"] is None else inputs["audio"][:n_s].cpu().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    ind = po.zone_indicator(v, 8, wl.H, wl.W, audio)
+    shape_id, base, blocks = po.assign_blocks(ind["g"], ind["rho"], 8, wl.H, wl.W)
+    perm = po.permutation(8, wl.H, wl.W, shape_id)
+    qp, kp, vp, dop = (po.permute(x, perm) for x in (q, k, v, do))
+    qbar, kbar = po.pool_blocks(qp, blocks), po.pool_blocks(kp, blocks)
+    t_prep = time.perf_counter() - t0
+    nb = len(blocks)
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    rng = np.random.default_rng(seed)
+    heads = sorted(rng.choice(wl.heads, size=min(2, wl.heads), replace=False).tolist())
+    per_head = {h: tuple(np.ascontiguousarray(x[h:h + 1], dtype=np.float64) for x in (qp, kp, vp, dop))
+                for h in heads}
+    step_vals = []
+    rows_done = 0
+    flops_total = 0.0
+    t_total = 0.0
+    per_step_budget = budget_s / max(1, steps)
+    for _ in range(steps):
+        t_step = 0.0
+        f_step = 0.0
+        while t_step < per_step_budget:
+            h, i = heads[int(rng.integers(len(heads)))], int(rng.integers(nb))
+            hq, hk, hv, hdo = per_head[h]
+            t1 = time.perf_counter()
+            s = po.block_scores(qbar[h][i:i + 1], kbar[h], scale)[0]
+            sel = po.select_row(po.block_probabilities(s), wl.top_k, wl.top_p)
+            row_ptr = np.zeros((1, nb + 1), dtype=np.int64)
+            row_ptr[0, i + 1:] = len(sel)
+            po.bsa_forward(hq, hk, hv, blocks, row_ptr, [sel], scale, query_blocks=[i])
+            po.bsa_backward(hq, hk, hv, hdo, blocks, row_ptr, [sel], scale, query_blocks=[i])
+            dt = time.perf_counter() - t1
+            t_step += dt
+            f_step += 14.0 * blocks[i][1] * float(blocks[sel, 1].sum()) * wl.head_dim
+            rows_done += 1
+        step_vals.append(f_step / t_step / 1e12)
+        flops_total += f_step
+        t_total += t_step
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    return dict(value=flops_total / t_total / 1e12, unit=UNIT, cores=cores, kind="oracle",
+                sample=(f"first 8-frame slab (8x{wl.H}x{wl.W}, {wl.heads} heads) of the {wl.name} inputs: "
+                        f"indicator/assign/permute/pool in full ({t_prep:.1f} s, not in the rate); "
+                        f"select+fwd+bwd on {rows_done} random query blocks of heads {heads}, fp64 numpy"),
+                step_values=step_vals, prep_s=t_prep, seconds=t_total)
+
+
+# ----------------------------------------------------------------- ranks --
+def setup_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ GPU bench --
+def run_prism(args, rank, world):
+    from dynamic_block_sparse_variance_b200 import prism as P
+    from dynamic_block_sparse_variance_b200 import synth
+    from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
+
+    P.lib()
+    wl = synth.get_workload(args.workload)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inputs = synth.make_inputs(wl, dev, with_dout=True)
+    att = PrismSparseAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, device=dev)
+    shp = (wl.N, wl.heads, wl.head_dim)
+    O = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+    dq, dk, dv = (torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(3))
+
+    def step():
+        att.forward(inputs["q"], inputs["k"], inputs["v"], inputs["audio"], out=O)
+        att.backward(inputs["dout"], dq, dk, dv)
+
+    for _ in range(args.warmup):
+        step()
+    P.prism_device_status()
+    pairs, nnz, nb, sizes = executed_pairs(att)
+    Punit = float(pairs) * wl.head_dim
+    exec_flops = 14.0 * Punit
+    dense_flops = 14.0 * float(wl.N) ** 2 * wl.head_dim * wl.heads
+
+    clocks = ClockSampler(dev)
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    with P.KernelTrace() as tr:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    P.prism_device_status()
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = max_over_ranks(ms_local, world)
+    summ = tr.summary()
+    launches = sum(n for n, _ in summ.values())
+
+    # dominant kernel and its roofline
+    peaks, peak_src = load_peaks()
+    dom = max(summ.items(), key=lambda kv: kv[1][1])
+    dom_name, (dom_n, dom_ms) = dom
+    if dom_name in KERNEL_FLOP_UNITS:
+        per_launch = KERNEL_FLOP_UNITS[dom_name] * Punit
+        achieved = per_launch / (dom_ms / dom_n * 1e-3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        roof = dict(kernel=dom_name, bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
+                    frac=achieved / peak, traffic=None, peak_source=f"{peak_src} sustained bf16 (cuBLAS)",
+                    flops_per_launch=per_launch, ms_per_launch=dom_ms / dom_n)
+    else:
+        roof = dict(kernel=dom_name, bound="hbm", achieved=None, peak=peaks.get("hbm_gbs"), unit="GB/s",
+                    frac=None, traffic=None)
+    t_fwd = summ.get("bsa_fwd_mma_kernel", (0, 0.0))[1] / args.steps
+    t_bwd = sum(summ.get(k, (0, 0.0))[1] for k in ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel")) / args.steps
+    burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    value = world * exec_flops / (ms * 1e-3) / 1e12
+    out = dict(
+        metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+        ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
+        data="synthetic",
+        config=dict(workload=f"{wl.name}-like grid {wl.T}x{wl.H}x{wl.W}", T=wl.T, H=wl.H, W=wl.W, N=wl.N,
+                    heads=wl.heads, head_dim=wl.head_dim, top_k=wl.top_k, top_p=wl.top_p,
+                    l2="inputs larger than L2 (each Q/K/V tensor %.2f GB)" % (wl.N * wl.heads * wl.head_dim * 2 / 1e9),
+                    parallelism=f"replicas x{world}"),
+        roofline=roof,
+        attention=dict(fwd_ms=t_fwd, bwd_ms=t_bwd, executed_tflop=exec_flops / 1e12,
+                       dense_equiv_tflop=dense_flops / 1e12,
+                       attn_executed_tflops=exec_flops / ((t_fwd + t_bwd) * 1e-3) / 1e12 if t_fwd + t_bwd else None,
+                       step_executed_pct_of_burst_peak=100.0 * exec_flops / (ms * 1e-3) / 1e12 / burst,
+                       dense_equiv_tflops=dense_flops / (ms * 1e-3) / 1e12,
+                       flop_density=pairs / (wl.heads * float(wl.N) ** 2),
+                       block_density=nnz / (wl.heads * float(nb) ** 2), nblk=nb, nnz=nnz,
+                       B_hist={int(b): int((sizes == b).sum().item()) for b in (64, 128, 256)}),
+        kernels={k: dict(launches=n, ms_per_step=t / args.steps) for k, (n, t) in sorted(summ.items())},
+        gpu_launches=launches,
+        clocks=clk,
+    )
+    # end-to-end through the public API with host buffers
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(att, inputs, (O, dq, dk, dv), wl, exec_flops, args, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = {k: v for k, v in oracle_sample(inputs, wl, args.cpu_budget_s).items()
+                               if k in ("value", "unit", "cores", "kind", "sample", "prep_s", "seconds")}
+    return out
+
+
+def run_e2e(att, inputs, outs, wl, exec_flops, args, world):
+    """Same step with inputs in pinned host memory: H2D of Q, K, V, audio, dO and
+    D2H of O, dQ, dK, dV inside the timed region (the device buffers of the
+    kernel-only run are reused as the copies' targets and sources)."""
+    names = ["q", "k", "v", "audio", "dout"]
+    host = {n: (None if inputs[n] is None else torch.empty(inputs[n].shape, dtype=inputs[n].dtype,
+                                                           pin_memory=True).copy_(inputs[n]))
+            for n in names}
+    out_host = torch.empty((wl.N, wl.heads, wl.head_dim), dtype=torch.bfloat16, pin_memory=True)
+    dev_in = inputs
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = 4 * out_host.numel() * out_host.element_size()
+
+    def step():
+        for n in names:
+            if host[n] is not None:
+                dev_in[n].copy_(host[n], non_blocking=True)
+        att.forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["audio"], out=outs[0])
+        att.backward(dev_in["dout"], outs[1], outs[2], outs[3])
+        for o in outs:
+            out_host.copy_(o, non_blocking=True)
+
+    step()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.e2e_steps, world)
+    return dict(value=world * exec_flops / (ms * 1e-3) / 1e12, unit=UNIT, ms_per_step=ms,
+                h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h, steps=args.e2e_steps)
+
+
+# ----------------------------------------------------- reference (oracle) --
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle on the host cores, on a bounded sample of the workload."""
+    if rank != 0:
+        return None
+    from dynamic_block_sparse_variance_b200 import synth
+
+    wl = synth.get_workload(args.workload)
+    gdev = "cuda" if torch.cuda.is_available() else "cpu"
+    inputs = synth.make_inputs(wl, gdev, with_dout=True)
+    budget = min(args.cpu_budget_s * max(1, args.steps), 150.0)
+    cb = oracle_sample(inputs, wl, budget, steps=max(1, args.steps))
+    value = cb["value"]
+    return dict(
+        metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
+        ms_per_step=cb["seconds"] * 1e3 / max(1, args.steps), higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
+        config=dict(workload=f"{wl.name}-like grid {wl.T}x{wl.H}x{wl.W}", T=wl.T, H=wl.H, W=wl.W,
+                    heads=wl.heads, head_dim=wl.head_dim, top_k=wl.top_k, top_p=wl.top_p,
+                    parallelism="host cores"),
+        cpu_baseline=dict(kind="oracle", cores=cb["cores"], sample=cb["sample"], value=value, unit=UNIT),
+        e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0),
+        gpu_launches=0,
+    )
+
+
+def main():
+    args = parse_args()
+    rank, world, _ = setup_dist(args)
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, rank, world)
+        else:
+            res = run_prism(args, rank, world)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -21,13 +21,15 @@ class PrismSparseAttention:
     Inputs are natural-layout [N, heads, head_dim] tensors (bf16, or f32 which
     the permutation rounds to bf16), N = T*H*W in raster order (t, y, x).
     ``col_capacity`` bounds the number of selected (query block, key block)
-    pairs over all heads; the default allows a quarter of all pairs.
+    pairs over all heads; the default allows every pair on small grids and a
+    quarter of them on large ones.  With ``training`` the forward also keeps
+    the bf16 rounding residual of O for the backward's row sums.
     ``select_ws_bytes`` bounds the block-score workspace (heads are processed
     in passes that fit).
     """
 
     def __init__(self, T, H, W, heads, head_dim, top_k, top_p, *, tau128=0.5, tau256=0.25, eps=1e-4,
-                 scale=0.0, col_capacity=None, select_ws_bytes=4 << 30, device="cuda"):
+                 scale=0.0, col_capacity=None, select_ws_bytes=4 << 30, training=True, device="cuda"):
         self.p = P.make_params(T, H, W, heads, head_dim, top_k, top_p, tau128, tau256, eps, scale)
         self.T, self.H, self.W, self.heads, self.D = T, H, W, heads, head_dim
         self.N = T * H * W
@@ -48,12 +50,14 @@ class PrismSparseAttention:
         self.kp = torch.empty_like(self.qp)
         self.vp = torch.empty_like(self.qp)
         self.op = torch.empty_like(self.qp)
+        self.op_res = torch.empty_like(self.qp) if training else None
         self.qbar = torch.empty(heads, cap, D, dtype=f32, device=dev)
         self.kbar = torch.empty_like(self.qbar)
         self.lse = torch.empty(heads, N, dtype=f32, device=dev)
         self.row_ptr = torch.empty(heads * cap + 1, dtype=i32, device=dev)
         if col_capacity is None:
-            col_capacity = min(heads * cap * cap // 4, 2**31 - 1)
+            pairs = heads * cap * cap
+            col_capacity = min(pairs, max(1 << 24, pairs // 4), 2**31 - 1)
         self.col = torch.empty(int(col_capacity), dtype=i32, device=dev)
         self.nnz = torch.empty(1, dtype=torch.int64, device=dev)
         ind, _ = P.prism_workspace_size(self.p, P.PRISM_WS_INDICATOR)
@@ -80,7 +84,7 @@ class PrismSparseAttention:
 
     def attend(self):
         P.prism_bsa_fwd(self.p, self.blocks, self.zone_blk_base, self.nblk, self.qp, self.kp, self.vp,
-                        self.row_ptr, self.col, self.op, self.lse)
+                        self.row_ptr, self.col, self.op, self.lse, o_res=self.op_res)
 
     def forward(self, q, k, v, audio=None, out=None):
         """Natural-layout output O [N, heads, head_dim] bf16."""
@@ -106,7 +110,7 @@ class PrismSparseAttention:
     def attend_backward(self):
         b = self._bwd_buffers()
         P.prism_bsa_bwd(self.p, self.blocks, self.zone_blk_base, self.nblk, self.qp, self.kp, self.vp, self.op,
-                        b["dop"], self.lse, self.row_ptr, self.col, self.nnz, b["dqp"], b["dkp"], b["dvp"],
+                        self.op_res, b["dop"], self.lse, self.row_ptr, self.col, self.nnz, b["dqp"], b["dkp"], b["dvp"],
                         b["ws"])
 
     def backward(self, dout, dq=None, dk=None, dv=None):

@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(128) bsa_fwd_mma_kernel(
     const __nv_bfloat16 *__restrict__ v, const prism_block *__restrict__ blocks,
     const int32_t *__restrict__ zone_blk_base, const int32_t *__restrict__ row_ptr,
     const int32_t *__restrict__ col, int64_t N, int64_t cap, float scale_log2,
-    __nv_bfloat16 *__restrict__ o, float *__restrict__ lse) {
+    __nv_bfloat16 *__restrict__ o, __nv_bfloat16 *__restrict__ o_res, float *__restrict__ lse) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int TILE = 64 * D * 2;
   const uint32_t sQ = smem_u32(smem), sK = sQ + TILE, sV = sQ + 3 * TILE;
@@ -163,8 +163,14 @@ __global__ void __launch_bounds__(128) bsa_fwd_mma_kernel(
 #pragma unroll
   for (int t = 0; t < D / 8; ++t) {
     const int c = t * 8 + (lane & 3) * 2;
-    *reinterpret_cast<uint32_t *>(oa + c) = pack_bf16(acc[t][0] * inv0, acc[t][1] * inv0);
-    *reinterpret_cast<uint32_t *>(ob + c) = pack_bf16(acc[t][2] * inv1, acc[t][3] * inv1);
+    const float x0 = acc[t][0] * inv0, x1 = acc[t][1] * inv0, x2 = acc[t][2] * inv1, x3 = acc[t][3] * inv1;
+    const uint32_t ua = pack_bf16(x0, x1), ub = pack_bf16(x2, x3);
+    *reinterpret_cast<uint32_t *>(oa + c) = ua;
+    *reinterpret_cast<uint32_t *>(ob + c) = ub;
+    if (o_res) {
+      *reinterpret_cast<uint32_t *>(o_res + hoff + ra * D + c) = pack_bf16(x0 - bf16_lo(ua), x1 - bf16_hi(ua));
+      *reinterpret_cast<uint32_t *>(o_res + hoff + rb * D + c) = pack_bf16(x2 - bf16_lo(ub), x3 - bf16_hi(ub));
+    }
   }
   if ((lane & 3) == 0) {
     lse[(int64_t)h * N + ra] = lrow[0] > 0.f ? (mrow[0] + log2f(lrow[0])) * kLn2 : -INFINITY;

@@ -1,6 +1,7 @@
 // Backward of the block-sparse attention on the warp-level bf16 MMA.
 //
-// bwd_delta_kernel   D_r = sum_c dO_rc O_rc (fp32), one warp per row.
+// bwd_delta_kernel   D_r = sum_c dO_rc O_rc (fp32), one warp per row; O is the
+//                    bf16 output plus, when given, its rounding residual.
 // csc kernels        transpose of the selection (per head, key block ->
 //                    ascending query blocks), so dK/dV are owned by one CTA.
 // bsa_dkdv_mma_kernel  one CTA per (64-key tile, head): walks the query blocks
@@ -16,6 +17,7 @@ namespace prism {
 
 template <int D>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16 *__restrict__ o,
+                                                        const __nv_bfloat16 *__restrict__ o_res,
                                                         const __nv_bfloat16 *__restrict__ dout,
                                                         int64_t rows, float *__restrict__ delta) {
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -28,7 +30,13 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16 *__r
   for (int e = 0; e < PER; e += 2) {
     const uint32_t ua = *reinterpret_cast<const uint32_t *>(a + e);
     const uint32_t ub = *reinterpret_cast<const uint32_t *>(b + e);
-    s += bf16_lo(ua) * bf16_lo(ub) + bf16_hi(ua) * bf16_hi(ub);
+    float o0 = bf16_lo(ua), o1 = bf16_hi(ua);
+    if (o_res) {
+      const uint32_t ur = *reinterpret_cast<const uint32_t *>(o_res + r * D + lane * PER + e);
+      o0 += bf16_lo(ur);
+      o1 += bf16_hi(ur);
+    }
+    s += o0 * bf16_lo(ub) + o1 * bf16_hi(ub);
   }
   s = warp_sum(s);
   if (lane == 0) delta[r] = s;

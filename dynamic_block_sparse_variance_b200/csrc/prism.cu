@@ -13,6 +13,25 @@
 namespace prism {
 
 static thread_local std::string t_error;
+static prism_trace_fn g_trace = nullptr;
+static void *g_trace_user = nullptr;
+
+// Brackets one kernel launch with the trace hook (if any).
+struct TraceScope {
+  const char *name;
+  cudaStream_t st;
+  TraceScope(const char *n, cudaStream_t s) : name(n), st(s) {
+    if (g_trace) g_trace(g_trace_user, name, 0, st);
+  }
+  ~TraceScope() {
+    if (g_trace) g_trace(g_trace_user, name, 1, st);
+  }
+};
+#define PRISM_TRACED(NAME, ST, ...) \
+  do {                              \
+    TraceScope _ts(NAME, ST);       \
+    __VA_ARGS__;                    \
+  } while (0)
 
 int fail(int code, const char *msg) {
   t_error = msg ? msg : "";
@@ -92,9 +111,9 @@ struct BwdWs {
 
 static int launch_scan(const int32_t *cnt, int64_t R, long long *part, int64_t nchunk, int64_t capacity,
                        int32_t *row_ptr, int64_t *nnz, cudaStream_t st) {
-  scan_partial_kernel<<<(unsigned)nchunk, kScanThreads, 0, st>>>(cnt, R, part);
-  scan_top_kernel<<<1, kScanThreads, 0, st>>>(part, (int)nchunk, capacity, nnz);
-  scan_final_kernel<<<(unsigned)nchunk, kScanThreads, 0, st>>>(cnt, R, part, nnz, capacity, row_ptr);
+  PRISM_TRACED("scan_partial_kernel", st, scan_partial_kernel<<<(unsigned)nchunk, kScanThreads, 0, st>>>(cnt, R, part));
+  PRISM_TRACED("scan_top_kernel", st, scan_top_kernel<<<1, kScanThreads, 0, st>>>(part, (int)nchunk, capacity, nnz));
+  PRISM_TRACED("scan_final_kernel", st, scan_final_kernel<<<(unsigned)nchunk, kScanThreads, 0, st>>>(cnt, R, part, nnz, capacity, row_ptr));
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
 }
@@ -106,6 +125,12 @@ using namespace prism;
 extern "C" {
 
 const char *prism_last_error(void) { return t_error.c_str(); }
+
+int prism_set_trace(prism_trace_fn fn, void *user) {
+  g_trace = fn;
+  g_trace_user = user;
+  return PRISM_OK;
+}
 
 int prism_device_status(prism_stream stream) {
   cudaError_t e = cudaStreamSynchronize(as_stream(stream));
@@ -164,13 +189,13 @@ int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, cons
   double *rec = reinterpret_cast<double *>(ws + w.rec);
   dim3 grid(w.nslab, (unsigned)d.Z);
   if (v_dtype == PRISM_BF16)
-    zone_stats_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(V), (int)d.C,
-                                                            d.H, d.W, d.ZY, d.ZX, part);
+    PRISM_TRACED("zone_stats_kernel", st, zone_stats_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(V), (int)d.C,
+                                                            d.H, d.W, d.ZY, d.ZX, part));
   else
-    zone_stats_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(V), (int)d.C, d.H, d.W, d.ZY,
-                                                    d.ZX, part);
-  zone_finish_kernel<<<(unsigned)d.Z, 64, 0, st>>>(part, w.nslab, (int)d.C, audio, d.H, d.W, d.ZY, d.ZX, rec);
-  zone_final_kernel<<<1, 1024, 0, st>>>(rec, (int)d.Z, audio != nullptr, p->eps, g, rho, debug);
+    PRISM_TRACED("zone_stats_kernel", st, zone_stats_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(V), (int)d.C, d.H, d.W, d.ZY,
+                                                    d.ZX, part));
+  PRISM_TRACED("zone_finish_kernel", st, zone_finish_kernel<<<(unsigned)d.Z, 64, 0, st>>>(part, w.nslab, (int)d.C, audio, d.H, d.W, d.ZY, d.ZX, rec));
+  PRISM_TRACED("zone_final_kernel", st, zone_final_kernel<<<1, 1024, 0, st>>>(rec, (int)d.Z, audio != nullptr, p->eps, g, rho, debug));
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
 }
@@ -182,8 +207,8 @@ int prism_assign_blocks(const prism_params *p, const float *g, const float *rho,
   if (rc) return rc;
   if (!g || !rho || !shape_id || !zone_blk_base || !blocks || !nblk)
     return fail(PRISM_EINVAL, "assign_blocks: NULL argument");
-  assign_blocks_kernel<<<1, 1024, 0, as_stream(stream)>>>(g, rho, (int)d.Z, p->tau128, p->tau256, shape_id,
-                                                          zone_blk_base, blocks, nblk);
+  PRISM_TRACED("assign_blocks_kernel", as_stream(stream), assign_blocks_kernel<<<1, 1024, 0, as_stream(stream)>>>(g, rho, (int)d.Z, p->tau128, p->tau256, shape_id,
+                                                          zone_blk_base, blocks, nblk));
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
 }
@@ -200,8 +225,8 @@ int prism_permute(const prism_params *p, const uint8_t *shape_id, const int32_t 
   dim3 grid(d.heads, (unsigned)d.Z);
   auto *xp = static_cast<__nv_bfloat16 *>(x_perm);
 #define PRISM_PERMUTE(TIN, DD)                                                                                \
-  permute_kernel<TIN, DD><<<grid, 256, 0, st>>>(static_cast<const TIN *>(x), d.heads, d.N, d.H, d.W, d.ZY, d.ZX, \
-                                                shape_id, zone_blk_base, d.cap, xp, pooled)
+  PRISM_TRACED("permute_kernel", st, permute_kernel<TIN, DD><<<grid, 256, 0, st>>>(static_cast<const TIN *>(x), d.heads, d.N, d.H, d.W, d.ZY, d.ZX, \
+                                                shape_id, zone_blk_base, d.cap, xp, pooled))
   if (x_dtype == PRISM_BF16) {
     if (d.D == 128) PRISM_PERMUTE(__nv_bfloat16, 128); else PRISM_PERMUTE(__nv_bfloat16, 64);
   } else {
@@ -224,8 +249,8 @@ int prism_unpermute(const prism_params *p, const uint8_t *shape_id, const void *
   cudaStream_t st = as_stream(stream);
   dim3 grid(d.heads, (unsigned)d.Z);
 #define PRISM_UNPERMUTE(TIN, TOUT, DD)                                                                        \
-  unpermute_kernel<TIN, TOUT, DD><<<grid, 256, 0, st>>>(static_cast<const TIN *>(x_perm), d.heads, d.N, d.H, \
-                                                        d.W, d.ZY, d.ZX, shape_id, static_cast<TOUT *>(x))
+  PRISM_TRACED("unpermute_kernel", st, unpermute_kernel<TIN, TOUT, DD><<<grid, 256, 0, st>>>(static_cast<const TIN *>(x_perm), d.heads, d.N, d.H, \
+                                                        d.W, d.ZY, d.ZX, shape_id, static_cast<TOUT *>(x)))
 #define PRISM_UNPERMUTE_D(TIN, TOUT) \
   do { if (d.D == 128) PRISM_UNPERMUTE(TIN, TOUT, 128); else PRISM_UNPERMUTE(TIN, TOUT, 64); } while (0)
   if (in_dtype == PRISM_BF16 && out_dtype == PRISM_BF16) PRISM_UNPERMUTE_D(__nv_bfloat16, __nv_bfloat16);
@@ -267,9 +292,9 @@ int prism_block_select(const prism_params *p, const int32_t *nblk, const float *
   cudaFuncSetAttribute(row_cut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)key_bytes);
   for (int h0 = 0; h0 < d.heads; h0 += hp) {
     const int nh = std::min(hp, d.heads - h0);
-    block_scores_kernel<<<dim3(tiles, tiles, nh), 256, 0, st>>>(q_pooled, k_pooled, d.D, d.cap, nblk, h0, scale, S);
-    row_cut_kernel<<<dim3((unsigned)d.cap, nh), kSelThreads, key_bytes, st>>>(S, d.cap, nblk, h0, p->top_k,
-                                                                               p->top_p, cnt, ckey, cq);
+    PRISM_TRACED("block_scores_kernel", st, block_scores_kernel<<<dim3(tiles, tiles, nh), 256, 0, st>>>(q_pooled, k_pooled, d.D, d.cap, nblk, h0, scale, S));
+    PRISM_TRACED("row_cut_kernel", st, row_cut_kernel<<<dim3((unsigned)d.cap, nh), kSelThreads, key_bytes, st>>>(S, d.cap, nblk, h0, p->top_k,
+                                                                               p->top_p, cnt, ckey, cq));
   }
   PRISM_CUDA_CHECK_LAUNCH();
   rc = launch_scan(cnt, w.R, part, w.nchunk, col_capacity, row_ptr, nnz, st);
@@ -277,9 +302,9 @@ int prism_block_select(const prism_params *p, const int32_t *nblk, const float *
   for (int h0 = 0; h0 < d.heads; h0 += hp) {
     const int nh = std::min(hp, d.heads - h0);
     if (!once)
-      block_scores_kernel<<<dim3(tiles, tiles, nh), 256, 0, st>>>(q_pooled, k_pooled, d.D, d.cap, nblk, h0, scale, S);
-    emit_kernel<<<dim3((unsigned)d.cap, nh), kSelThreads, 0, st>>>(S, d.cap, nblk, h0, ckey, cq, row_ptr, nnz,
-                                                                  col_capacity, col);
+      PRISM_TRACED("block_scores_kernel", st, block_scores_kernel<<<dim3(tiles, tiles, nh), 256, 0, st>>>(q_pooled, k_pooled, d.D, d.cap, nblk, h0, scale, S));
+    PRISM_TRACED("emit_kernel", st, emit_kernel<<<dim3((unsigned)d.cap, nh), kSelThreads, 0, st>>>(S, d.cap, nblk, h0, ckey, cq, row_ptr, nnz,
+                                                                  col_capacity, col));
   }
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
@@ -304,7 +329,7 @@ extern "C" {
 
 int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
                   const int32_t *nblk, const void *q, const void *k, const void *v, const int32_t *row_ptr,
-                  const int32_t *col, void *o, float *lse, void *workspace, size_t ws_bytes,
+                  const int32_t *col, void *o, void *o_res, float *lse, void *workspace, size_t ws_bytes,
                   prism_stream stream) {
   (void)workspace;
   (void)ws_bytes;
@@ -318,15 +343,17 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
   auto Q = static_cast<const __nv_bfloat16 *>(q), K = static_cast<const __nv_bfloat16 *>(k),
        Vv = static_cast<const __nv_bfloat16 *>(v);
   auto O = static_cast<__nv_bfloat16 *>(o);
+  auto Ores = static_cast<__nv_bfloat16 *>(o_res);
+  if (o_res && !aligned16(o_res)) return fail(PRISM_EINVAL, "attention: o_res must be 16-byte aligned");
   if (d.D == 128) {
     const int smem = 5 * 64 * 128 * 2;
     cudaFuncSetAttribute(bsa_fwd_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    bsa_fwd_mma_kernel<128><<<grid, 128, smem, st>>>(Q, K, Vv, blocks, zone_blk_base, row_ptr, col, d.N, d.cap,
-                                                     scale_log2, O, lse);
+    PRISM_TRACED("bsa_fwd_mma_kernel", st, bsa_fwd_mma_kernel<128><<<grid, 128, smem, st>>>(Q, K, Vv, blocks, zone_blk_base, row_ptr, col, d.N, d.cap,
+                                                     scale_log2, O, Ores, lse));
   } else {
     const int smem = 5 * 64 * 64 * 2;
-    bsa_fwd_mma_kernel<64><<<grid, 128, smem, st>>>(Q, K, Vv, blocks, zone_blk_base, row_ptr, col, d.N, d.cap,
-                                                    scale_log2, O, lse);
+    PRISM_TRACED("bsa_fwd_mma_kernel", st, bsa_fwd_mma_kernel<64><<<grid, 128, smem, st>>>(Q, K, Vv, blocks, zone_blk_base, row_ptr, col, d.N, d.cap,
+                                                    scale_log2, O, Ores, lse));
   }
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
@@ -345,17 +372,18 @@ static void launch_bwd_attn(const Dims &d, dim3 grid, cudaStream_t st, const __n
   const int smem_q = 6 * 64 * D * 2;
   cudaFuncSetAttribute(bsa_dkdv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_kv);
   cudaFuncSetAttribute(bsa_dq_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_q);
-  bsa_dkdv_mma_kernel<D><<<grid, 128, smem_kv, st>>>(Q, K, Vv, dO, lse, delta, blocks, zbb, col_ptr, row_idx,
-                                                      d.N, d.cap, scale, dk, dv);
-  bsa_dq_mma_kernel<D><<<grid, 128, smem_q, st>>>(Q, K, Vv, dO, lse, delta, blocks, zbb, row_ptr, col, d.N,
-                                                   d.cap, scale, dq);
+  PRISM_TRACED("bsa_dkdv_mma_kernel", st, bsa_dkdv_mma_kernel<D><<<grid, 128, smem_kv, st>>>(Q, K, Vv, dO, lse, delta, blocks, zbb, col_ptr, row_idx,
+                                                      d.N, d.cap, scale, dk, dv));
+  PRISM_TRACED("bsa_dq_mma_kernel", st, bsa_dq_mma_kernel<D><<<grid, 128, smem_q, st>>>(Q, K, Vv, dO, lse, delta, blocks, zbb, row_ptr, col, d.N,
+                                                   d.cap, scale, dq));
 }
 
 extern "C" {
 
 int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
                   const int32_t *nblk, const void *q, const void *k, const void *v, const void *o,
-                  const void *dout, const float *lse, const int32_t *row_ptr, const int32_t *col,
+                  const void *o_res, const void *dout, const float *lse, const int32_t *row_ptr,
+                  const int32_t *col,
                   const int64_t *nnz, int64_t col_capacity, void *dq, void *dk, void *dv, void *workspace,
                   size_t ws_bytes, prism_stream stream) {
   Dims d;
@@ -376,22 +404,24 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
   long long *part = reinterpret_cast<long long *>(ws + w.part);
   int32_t *row_idx = reinterpret_cast<int32_t *>(ws + w.row_idx);
   auto O = static_cast<const __nv_bfloat16 *>(o), dO = static_cast<const __nv_bfloat16 *>(dout);
+  auto Ores = static_cast<const __nv_bfloat16 *>(o_res);
+  if (o_res && !aligned16(o_res)) return fail(PRISM_EINVAL, "bwd: o_res must be 16-byte aligned");
   const int64_t rows = (int64_t)d.heads * d.N;
   if (d.D == 128)
-    bwd_delta_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, dO, rows, delta);
+    PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, rows, delta));
   else
-    bwd_delta_kernel<64><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, dO, rows, delta);
+    PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<64><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, rows, delta));
   cudaMemsetAsync(ccnt, 0, w.R * 4, st);
   cudaMemsetAsync(fill, 0, w.R * 4, st);
   dim3 rgrid((unsigned)d.cap, d.heads);
-  csc_count_kernel<<<rgrid, 256, 0, st>>>(row_ptr, col, d.cap, nblk, ccnt);
+  PRISM_TRACED("csc_count_kernel", st, csc_count_kernel<<<rgrid, 256, 0, st>>>(row_ptr, col, d.cap, nblk, ccnt));
   // column counts -> column pointers (their total equals the selection's nnz)
   int64_t *tot = reinterpret_cast<int64_t *>(ws + w.tot);
   rc = launch_scan(ccnt, w.R, part, w.nchunk, col_capacity, col_ptr, tot, st);
   if (rc) return rc;
-  csc_fill_kernel<<<rgrid, 256, 0, st>>>(row_ptr, col, d.cap, nblk, col_ptr, fill, row_idx);
+  PRISM_TRACED("csc_fill_kernel", st, csc_fill_kernel<<<rgrid, 256, 0, st>>>(row_ptr, col, d.cap, nblk, col_ptr, fill, row_idx));
   cudaFuncSetAttribute(csc_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sort_bytes);
-  csc_sort_kernel<<<rgrid, 512, sort_bytes, st>>>(col_ptr, d.cap, nblk, row_idx);
+  PRISM_TRACED("csc_sort_kernel", st, csc_sort_kernel<<<rgrid, 512, sort_bytes, st>>>(col_ptr, d.cap, nblk, row_idx));
   PRISM_CUDA_CHECK_LAUNCH();
   dim3 grid((unsigned)(d.N / 64), d.heads);
   auto Q = static_cast<const __nv_bfloat16 *>(q), K = static_cast<const __nv_bfloat16 *>(k),

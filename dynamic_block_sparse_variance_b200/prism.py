@@ -24,8 +24,10 @@ PRISM_WS_INDICATOR, PRISM_WS_SELECT, PRISM_WS_FWD, PRISM_WS_BWD = 0, 1, 2, 3
 ENTRY_POINTS = (
     "prism_workspace_size", "prism_zone_indicator", "prism_assign_blocks", "prism_permute",
     "prism_unpermute", "prism_block_select", "prism_bsa_fwd", "prism_bsa_bwd",
-    "prism_device_status", "prism_last_error",
+    "prism_set_trace", "prism_device_status", "prism_last_error",
 )
+
+TRACE_FN = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
 
 
 class PrismError(RuntimeError):
@@ -70,9 +72,10 @@ def lib():
             "prism_permute": [pp, _P, _P, _P, ctypes.c_int, _P, _P, _P],
             "prism_unpermute": [pp, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P],
             "prism_block_select": [pp, _P, _P, _P, _P, _P, i64, _P, _P, sz, _P],
-            "prism_bsa_fwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P],
-            "prism_bsa_bwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, i64, _P, _P, _P, _P,
-                              sz, _P],
+            "prism_bsa_fwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P],
+            "prism_bsa_bwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, i64, _P, _P, _P,
+                              _P, sz, _P],
+            "prism_set_trace": [TRACE_FN, _P],
             "prism_device_status": [_P],
             "prism_last_error": [],
         }
@@ -139,20 +142,58 @@ def prism_block_select(p, nblk, q_pooled, k_pooled, row_ptr, col, nnz, workspace
                                     _stream()))
 
 
-def prism_bsa_fwd(p, blocks, zone_blk_base, nblk, q, k, v, row_ptr, col, o, lse, workspace=None):
+def prism_bsa_fwd(p, blocks, zone_blk_base, nblk, q, k, v, row_ptr, col, o, lse, o_res=None, workspace=None):
     _check(lib().prism_bsa_fwd(ctypes.byref(p), _ptr(blocks), _ptr(zone_blk_base), _ptr(nblk), _ptr(q), _ptr(k),
-                               _ptr(v), _ptr(row_ptr), _ptr(col), _ptr(o), _ptr(lse), _ptr(workspace),
-                               0 if workspace is None else workspace.numel(), _stream()))
+                               _ptr(v), _ptr(row_ptr), _ptr(col), _ptr(o), _ptr(o_res), _ptr(lse),
+                               _ptr(workspace), 0 if workspace is None else workspace.numel(), _stream()))
 
 
-def prism_bsa_bwd(p, blocks, zone_blk_base, nblk, q, k, v, o, dout, lse, row_ptr, col, nnz, dq, dk, dv,
+def prism_bsa_bwd(p, blocks, zone_blk_base, nblk, q, k, v, o, o_res, dout, lse, row_ptr, col, nnz, dq, dk, dv,
                   workspace):
     _check(lib().prism_bsa_bwd(ctypes.byref(p), _ptr(blocks), _ptr(zone_blk_base), _ptr(nblk), _ptr(q),
-                               _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(row_ptr), _ptr(col),
-                               _ptr(nnz), col.numel(), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(workspace),
-                               workspace.numel(), _stream()))
+                               _ptr(k), _ptr(v), _ptr(o), _ptr(o_res), _ptr(dout), _ptr(lse), _ptr(row_ptr),
+                               _ptr(col), _ptr(nnz), col.numel(), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(workspace), workspace.numel(), _stream()))
 
 
 def prism_device_status():
     """Synchronise the current stream and raise if a kernel latched an error."""
     _check(lib().prism_device_status(_stream()))
+
+
+class KernelTrace:
+    """Records a CUDA event pair around every kernel the library launches.
+
+    Use as a context manager; ``summary()`` (after a synchronize) gives, per
+    kernel name, the number of launches and their total device time in ms.
+    """
+
+    def __init__(self):
+        self.events = []          # (name, start_event, end_event)
+        self._open = {}
+        self._cb = TRACE_FN(self._hook)
+
+    def _hook(self, user, name, end, stream):
+        s = torch.cuda.ExternalStream(stream) if stream else torch.cuda.default_stream()
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(s)
+        key = name.decode()
+        if not end:
+            self._open[key] = ev
+        else:
+            self.events.append((key, self._open.pop(key), ev))
+
+    def __enter__(self):
+        _check(lib().prism_set_trace(self._cb, None))
+        return self
+
+    def __exit__(self, *exc):
+        lib().prism_set_trace(TRACE_FN(), None)
+        return False
+
+    def summary(self):
+        out = {}
+        for name, a, b in self.events:
+            n, t = out.get(name, (0, 0.0))
+            out[name] = (n + 1, t + a.elapsed_time(b))
+        return out

@@ -180,18 +180,23 @@ int prism_block_select(const prism_params *p, const int32_t *nblk, const float *
  *   q, k, v               permuted [heads, N, head_dim] bf16, 16-B aligned
  *   row_ptr, col          CSR from prism_block_select
  *   o                     out permuted [heads, N, head_dim] bf16
+ *   o_res                 out, nullable: permuted [heads, N, head_dim] bf16, the
+ *                         rounding residual O_fp32 - O_bf16.  Training passes it
+ *                         to prism_bsa_bwd so that D = rowsum(dO o O) sees O to
+ *                         about 16 significant bits instead of 8.
  *   lse                   out [heads, N] float
  */
 int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
                   const int32_t *nblk, const void *q, const void *k, const void *v,
-                  const int32_t *row_ptr, const int32_t *col, void *o, float *lse, void *workspace,
-                  size_t ws_bytes, prism_stream stream);
+                  const int32_t *row_ptr, const int32_t *col, void *o, void *o_res, float *lse,
+                  void *workspace, size_t ws_bytes, prism_stream stream);
 
 /*
  * Backward of prism_bsa_fwd for the fixed selection: with P the attention
  * probabilities, dV = P^T dO, dP = dO V^T, D_r = rowsum(dO o O),
  * dS = P (dP - D), dQ = scale dS K, dK = scale dS^T Q.
  *   o, dout               permuted [heads, N, head_dim] bf16 (forward output, its gradient)
+ *   o_res                 nullable: the residual written by prism_bsa_fwd
  *   lse                   [heads, N] float from prism_bsa_fwd
  *   nnz, col_capacity     as returned to / given to prism_block_select
  *   dq, dk, dv            out permuted [heads, N, head_dim] bf16
@@ -199,9 +204,18 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
  */
 int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
                   const int32_t *nblk, const void *q, const void *k, const void *v, const void *o,
-                  const void *dout, const float *lse, const int32_t *row_ptr, const int32_t *col,
+                  const void *o_res, const void *dout, const float *lse, const int32_t *row_ptr, const int32_t *col,
                   const int64_t *nnz, int64_t col_capacity, void *dq, void *dk, void *dv,
                   void *workspace, size_t ws_bytes, prism_stream stream);
+
+/* Kernel-launch trace hook.  When set, the library calls
+ *   fn(user, kernel_name, 0, stream) just before and
+ *   fn(user, kernel_name, 1, stream) just after
+ * every kernel it launches, on the calling thread, so that a caller can
+ * record CUDA events around each kernel and count launches.  NULL disables.
+ * The hook is process-wide; set it while no other thread is calling in. */
+typedef void (*prism_trace_fn)(void *user, const char *kernel, int end, prism_stream stream);
+int prism_set_trace(prism_trace_fn fn, void *user);
 
 /* Synchronises `stream`, returns the latched device status (PRISM_OK or one
  * of PRISM_ECAPACITY / PRISM_ETIMEOUT / PRISM_EBOUNDS) and clears it. */

@@ -349,7 +349,7 @@ def bsa_forward(q, k, v, blocks, row_ptr, cols, scale, query_blocks=None, heads=
     return O, L
 
 
-def bsa_backward(q, k, v, dout, blocks, row_ptr, cols, scale):
+def bsa_backward(q, k, v, dout, blocks, row_ptr, cols, scale, query_blocks=None, heads=None):
     """Exact gradient of bsa_forward with respect to q, k, v for fixed S_i.
 
     The selection carries no gradient (it is discrete).  With
@@ -358,6 +358,8 @@ def bsa_backward(q, k, v, dout, blocks, row_ptr, cols, scale):
       dS_rc = P_rc (dP_rc - D_r),  dQ_r = scale sum_c dS_rc k_c,
       dK_c += scale sum_r dS_rc q_r.
     All arrays [heads, N, d] permuted; returns (dq, dk, dv) in float64.
+    query_blocks / heads restrict the sum to a sample of query blocks (dK, dV
+    then hold only those blocks' contributions).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -367,8 +369,8 @@ def bsa_backward(q, k, v, dout, blocks, row_ptr, cols, scale):
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
     Hh = q.shape[0]
-    for h in range(Hh):
-        for i in range(len(blocks)):
+    for h in (range(Hh) if heads is None else heads):
+        for i in (range(len(blocks)) if query_blocks is None else query_blocks):
             start, size = blocks[i][0], blocks[i][1]
             sel = cols[h][row_ptr[h, i]:row_ptr[h, i + 1]]
             rows = _key_rows(blocks, sel)
