@@ -68,10 +68,10 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         try:
-            bus = torch.cuda.get_device_properties(device).pci_bus_id
-            self.target = ["-i", bus]
+            pr = torch.cuda.get_device_properties(device)
+            self.target = ["-i", "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)]
         except Exception:
-            self.target = ["-i", str(torch.cuda.current_device())]
+            self.target = []
 
     def start(self):
         try:
@@ -122,7 +122,10 @@ def executed_pairs(att):
 # P = sum_h sum_i sum_{j in S_i} B_i B_j d: forward 4P (QK^T, PV); the key-side
 # backward kernel 8P (S, dP, dV, dK); the query-side one 2P (dQ; its S and dP
 # recomputation is extra work and not counted).
-KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_dkdv_mma_kernel": 8, "bsa_dq_mma_kernel": 2}
+KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_fwd_tc_kernel": 4, "bsa_dkdv_mma_kernel": 8,
+                     "bsa_dq_mma_kernel": 2}
+FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel")
+BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel")
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -286,8 +289,8 @@ def run_prism(args, rank, world):
     else:
         roof = dict(kernel=dom_name, bound="hbm", achieved=None, peak=peaks.get("hbm_gbs"), unit="GB/s",
                     frac=None, traffic=None)
-    t_fwd = summ.get("bsa_fwd_mma_kernel", (0, 0.0))[1] / args.steps
-    t_bwd = sum(summ.get(k, (0, 0.0))[1] for k in ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel")) / args.steps
+    t_fwd = sum(summ.get(k, (0, 0.0))[1] for k in FWD_KERNELS) / args.steps
+    t_bwd = sum(summ.get(k, (0, 0.0))[1] for k in BWD_KERNELS) / args.steps
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     value = world * exec_flops / (ms * 1e-3) / 1e12
     out = dict(

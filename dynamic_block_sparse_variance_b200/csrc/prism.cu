@@ -1,11 +1,14 @@
 // C ABI of the Prism sparse-attention library (declared in include/prism.h).
 // The whole library is this one translation unit: it includes the kernel
 // headers, validates arguments on the host, lays out workspaces and launches.
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <cstdio>
 #include <string>
 
 #include "attn_mma_bwd.cuh"
+#include "attn_tc_fwd.cuh"
 #include "indicator.cuh"
 #include "permute.cuh"
 #include "select.cuh"
@@ -13,6 +16,37 @@
 namespace prism {
 
 static thread_local std::string t_error;
+static int g_attn_backend = 0;
+static uint32_t g_wait_limit = 0;
+static int g_debug_stall = 0;
+constexpr uint32_t kDefaultWaitLimit = 1u << 22;
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [rows, 128] bf16 tensor, 64 x 128 boxes, 128-byte swizzle;
+// rows past the end read as zero.
+static bool make_tile_map(CUtensorMap *map, const void *base, uint64_t rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {128, rows};
+  cuuint64_t strides[1] = {128 * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 static prism_trace_fn g_trace = nullptr;
 static void *g_trace_user = nullptr;
 
@@ -125,6 +159,15 @@ using namespace prism;
 extern "C" {
 
 const char *prism_last_error(void) { return t_error.c_str(); }
+
+int prism_set_option(int option, int64_t value) {
+  switch (option) {
+    case PRISM_OPT_ATTN_BACKEND: g_attn_backend = (int)value; return PRISM_OK;
+    case PRISM_OPT_WAIT_LIMIT: g_wait_limit = (uint32_t)value; return PRISM_OK;
+    case PRISM_OPT_DEBUG_STALL: g_debug_stall = (int)value; return PRISM_OK;
+    default: return fail(PRISM_EINVAL, "unknown option");
+  }
+}
 
 int prism_set_trace(prism_trace_fn fn, void *user) {
   g_trace = fn;
@@ -345,7 +388,28 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
   auto O = static_cast<__nv_bfloat16 *>(o);
   auto Ores = static_cast<__nv_bfloat16 *>(o_res);
   if (o_res && !aligned16(o_res)) return fail(PRISM_EINVAL, "attention: o_res must be 16-byte aligned");
-  if (d.D == 128) {
+  if (d.D == 128 && g_attn_backend == 0) {
+    CUtensorMap tq, tk, tv;
+    const uint64_t rows = (uint64_t)d.heads * d.N;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
+      return fail(PRISM_ECUDA, "cuTensorMapEncodeTiled failed");
+    TcFwdArgs a;
+    a.blocks = blocks;
+    a.zone_blk_base = zone_blk_base;
+    a.row_ptr = row_ptr;
+    a.col = col;
+    a.N = d.N;
+    a.cap = d.cap;
+    a.scale_log2 = scale_log2;
+    a.o = O;
+    a.o_res = Ores;
+    a.lse = lse;
+    a.wait_limit = g_wait_limit ? g_wait_limit : kDefaultWaitLimit;
+    a.debug_stall = g_debug_stall;
+    cudaFuncSetAttribute(bsa_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
+    dim3 tgrid((unsigned)(d.Z * 8), d.heads);
+    PRISM_TRACED("bsa_fwd_tc_kernel", st, bsa_fwd_tc_kernel<<<tgrid, 192, kTcSmemBytes, st>>>(tq, tk, tv, a));
+  } else if (d.D == 128) {
     const int smem = 5 * 64 * 128 * 2;
     cudaFuncSetAttribute(bsa_fwd_mma_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     PRISM_TRACED("bsa_fwd_mma_kernel", st, bsa_fwd_mma_kernel<128><<<grid, 128, smem, st>>>(Q, K, Vv, blocks, zone_blk_base, row_ptr, col, d.N, d.cap,

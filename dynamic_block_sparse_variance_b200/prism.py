@@ -19,12 +19,13 @@ LIB_PATH = os.path.join(_HERE, "libprism_b200.so")
 PRISM_OK, PRISM_EINVAL, PRISM_ECAPACITY, PRISM_ECUDA, PRISM_ETIMEOUT, PRISM_EBOUNDS = 0, -1, -2, -3, -4, -5
 PRISM_BF16, PRISM_F32 = 0, 1
 PRISM_WS_INDICATOR, PRISM_WS_SELECT, PRISM_WS_FWD, PRISM_WS_BWD = 0, 1, 2, 3
+PRISM_OPT_ATTN_BACKEND, PRISM_OPT_WAIT_LIMIT, PRISM_OPT_DEBUG_STALL = 0, 1, 2
 
 # Entry points declared in include/prism.h, in declaration order.
 ENTRY_POINTS = (
     "prism_workspace_size", "prism_zone_indicator", "prism_assign_blocks", "prism_permute",
     "prism_unpermute", "prism_block_select", "prism_bsa_fwd", "prism_bsa_bwd",
-    "prism_set_trace", "prism_device_status", "prism_last_error",
+    "prism_set_option", "prism_set_trace", "prism_device_status", "prism_last_error",
 )
 
 TRACE_FN = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
@@ -75,6 +76,7 @@ def lib():
             "prism_bsa_fwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P],
             "prism_bsa_bwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, i64, _P, _P, _P,
                               _P, sz, _P],
+            "prism_set_option": [ctypes.c_int, i64],
             "prism_set_trace": [TRACE_FN, _P],
             "prism_device_status": [_P],
             "prism_last_error": [],
@@ -154,6 +156,10 @@ def prism_bsa_bwd(p, blocks, zone_blk_base, nblk, q, k, v, o, o_res, dout, lse, 
                                _ptr(k), _ptr(v), _ptr(o), _ptr(o_res), _ptr(dout), _ptr(lse), _ptr(row_ptr),
                                _ptr(col), _ptr(nnz), col.numel(), _ptr(dq), _ptr(dk), _ptr(dv),
                                _ptr(workspace), workspace.numel(), _stream()))
+
+
+def prism_set_option(option, value):
+    _check(lib().prism_set_option(option, value))
 
 
 def prism_device_status():

@@ -208,6 +208,21 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
                   const int64_t *nnz, int64_t col_capacity, void *dq, void *dk, void *dv,
                   void *workspace, size_t ws_bytes, prism_stream stream);
 
+/* Process-wide options (host-only; set while no call is in flight).
+ *   PRISM_OPT_ATTN_BACKEND  0 (default): tcgen05/TMEM/TMA attention kernels for
+ *                           head_dim 128, warp-level MMA kernels otherwise;
+ *                           1: warp-level MMA kernels always (cross-checking).
+ *   PRISM_OPT_WAIT_LIMIT    polls before a device-side wait gives up and
+ *                           latches PRISM_ETIMEOUT; 0 restores the default.
+ *   PRISM_OPT_DEBUG_STALL   test hook: when 1 the forward kernel never signals
+ *                           its first probability tile, so its bounded wait
+ *                           must time out (PRISM_ETIMEOUT), with no trap or hang.
+ * Returns PRISM_EINVAL for an unknown option. */
+#define PRISM_OPT_ATTN_BACKEND 0
+#define PRISM_OPT_WAIT_LIMIT 1
+#define PRISM_OPT_DEBUG_STALL 2
+int prism_set_option(int option, int64_t value);
+
 /* Kernel-launch trace hook.  When set, the library calls
  *   fn(user, kernel_name, 0, stream) just before and
  *   fn(user, kernel_name, 1, stream) just after

@@ -244,3 +244,25 @@ def test_capacity_overflow_is_reported_and_safe():
     assert int(att.nnz.item()) > 4
     assert int(att.row_ptr.max().item()) == 0     # every row left empty
     P.prism_device_status()                       # cleared
+
+
+def test_tc_forward_matches_warp_mma_forward():
+    """The tcgen05 forward (default for head_dim 128) and the warp-level MMA
+    forward agree on the same layout and selection (both are also checked
+    against the oracle above)."""
+    wl, inp, ora = problem("mix16")
+    outs = []
+    for backend in (0, 1):
+        P.prism_set_option(P.PRISM_OPT_ATTN_BACKEND, backend)
+        try:
+            att = make_att(wl)
+            _oracle_layout_on_gpu(att, ora, inp, wl)
+            att.attend()
+            P.prism_device_status()
+            outs.append((att.op.float().cpu(), att.lse.cpu(), att.op_res.float().cpu()))
+        finally:
+            P.prism_set_option(P.PRISM_OPT_ATTN_BACKEND, 0)
+    (o0, l0, r0), (o1, l1, r1) = outs
+    assert float((o0 - o1).abs().max()) <= 2e-2
+    assert float((l0 - l1).abs().max()) <= 1e-3
+    assert float(((o0 + r0) - (o1 + r1)).abs().max()) <= 1e-2

@@ -373,3 +373,18 @@ def test_pipeline_runs_end_to_end_with_every_volume():
     assert B[:8] == [64] * 8 and B[8:12] == [128] * 4 and set(B[12:]) == {256}
     assert out["O"].shape == (N, 2, 8) and np.isfinite(out["O"]).all()
     assert out["zone_blk_base"][-1] == len(out["blocks"])
+
+
+def test_bf16_half_ulp_helper():
+    """The tolerance helper is half the bf16 spacing: rounding any value to bf16
+    moves it by at most that much, and consecutive bf16 values above a
+    representable x differ by twice that."""
+    from tests.helpers import bf16_half_ulp
+    rng = np.random.default_rng(40)
+    x = rng.standard_normal(10000) * np.exp(rng.uniform(-5, 5, 10000))
+    r = torch.from_numpy(x).to(torch.bfloat16).double().numpy()
+    assert np.all(np.abs(r - x) <= bf16_half_ulp(x) * (1 + 1e-12))
+    for v in (1.0, 1.5, 3.0, 8.0, 9.5):
+        b = torch.tensor(v, dtype=torch.bfloat16)
+        nxt = torch.tensor(v + 2 * bf16_half_ulp(v), dtype=torch.bfloat16)
+        assert float(nxt) - float(b) == 2 * bf16_half_ulp(v)
