@@ -123,9 +123,9 @@ def executed_pairs(att):
 # backward kernel 8P (S, dP, dV, dK); the query-side one 2P (dQ; its S and dP
 # recomputation is extra work and not counted).
 KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_fwd_tc_kernel": 4, "bsa_dkdv_mma_kernel": 8,
-                     "bsa_dq_mma_kernel": 2}
+                     "bsa_dkdv_tc_kernel": 8, "bsa_dq_mma_kernel": 2, "bsa_dq_tc_kernel": 2}
 FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel")
-BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel")
+BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel", "bsa_dkdv_tc_kernel", "bsa_dq_tc_kernel")
 
 
 # ------------------------------------------------------------ CPU oracle --

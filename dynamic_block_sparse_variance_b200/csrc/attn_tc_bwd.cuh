@@ -1,0 +1,519 @@
+// Block-sparse attention backward on the tcgen05 tensor cores (head_dim 128).
+//
+// Two kernels, each owning its outputs, so the gradients need no atomics and
+// are bit-reproducible:
+//
+// bsa_dq_tc_kernel    one CTA per (128-row query tile, head), walking S_i:
+//   S_n = Q K_n^T and dP_n = dO V_n^T into tensor memory; one thread per query
+//   row turns them into dS = P (dP - D) with P = exp2(S log2e scale - LSE log2e),
+//   written as bf16 over S; dQ += dS K_n with dS read from tensor memory.
+//   TMEM: S0 | S1 | dP | dQ (4 x 128 columns).
+//
+// bsa_dkdv_tc_kernel  one CTA per (128-key tile, head), walking the query
+//   blocks that selected its key block (the transposed selection):
+//   S^T = K Q_n^T and dP^T = V dO_n^T into tensor memory; one thread per key
+//   row computes P^T (written back over S^T, the A operand of dV += P^T dO_n)
+//   and dS^T (written to 128-byte-swizzled shared memory, the A operand of
+//   dK += dS^T Q_n).  TMEM: dK | dV | S^T | dP^T.
+//
+// Roles, bounded waits and the abort path follow the forward kernel.
+#pragma once
+
+#include "attn_tc_fwd.cuh"
+
+namespace prism {
+
+struct TcBwdArgs {
+  const prism_block *blocks;
+  const int32_t *zone_blk_base;
+  const int32_t *row_ptr;   // dq: selection CSR
+  const int32_t *col;
+  const int32_t *col_ptr;   // dkdv: transposed selection
+  const int32_t *row_idx;
+  const float *lse;
+  const float *delta;
+  int64_t N, cap;
+  float scale_log2, scale;
+  __nv_bfloat16 *dq, *dk, *dv;
+  uint32_t wait_limit;
+};
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Tile of a zone: 128 rows (blocks of 128/256) or 64 rows (blocks of 64).
+struct ZoneTile {
+  int blk, r0, rows;
+  __device__ __forceinline__ bool init(const prism_block *blocks, const int32_t *zbb, int m, int t) {
+    const int b0 = zbb[m];
+    const int B = blocks[b0].size;
+    if (B >= 128 && t >= 4) return false;
+    if (B == 64) {
+      blk = b0 + t;
+      r0 = m * kZoneTokens + 64 * t;
+      rows = 64;
+    } else {
+      r0 = m * kZoneTokens + 128 * t;
+      blk = b0 + (128 * t) / B;
+      rows = 128;
+    }
+    return true;
+  }
+};
+
+// ============================================================================ dQ
+constexpr int kDqKStages = 3, kDqVStages = 2;
+constexpr int kDqSmemBytes = kTcTileBytes * (2 + kDqKStages + kDqVStages) + 256 + 1024;
+
+__global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                           const __grid_constant__ CUtensorMap tmK,
+                                                           const __grid_constant__ CUtensorMap tmV,
+                                                           const __grid_constant__ CUtensorMap tmO,
+                                                           const TcBwdArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t *sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t sQ = sbase, sO = sbase + kTcTileBytes;
+  auto sK = [&](int s) { return sbase + (uint32_t)(2 + s) * kTcTileBytes; };
+  auto sV = [&](int s) { return sbase + (uint32_t)(2 + kDqKStages + s) * kTcTileBytes; };
+  const uint32_t sBar = sbase + (uint32_t)(2 + kDqKStages + kDqVStages) * kTcTileBytes;
+  const uint32_t b_q = sBar;
+  auto b_kfull = [&](int s) { return sBar + 8u * (1 + s); };    // 3
+  auto b_kempty = [&](int s) { return sBar + 8u * (4 + s); };   // 3
+  auto b_vfull = [&](int s) { return sBar + 8u * (7 + s); };    // 2
+  auto b_vempty = [&](int s) { return sBar + 8u * (9 + s); };   // 2
+  auto b_sd = [&](int b) { return sBar + 8u * (11 + b); };      // S_n and dP_n done
+  auto b_ds = [&](int b) { return sBar + 8u * (13 + b); };      // dS_n written (128 arrivals)
+  const uint32_t b_drain = sBar + 8u * 15;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 16);
+  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 16 + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  ZoneTile zt;
+  if (!zt.init(args.blocks, args.zone_blk_base, blockIdx.x >> 3, blockIdx.x & 7)) return;
+  const int e0 = args.row_ptr[(int64_t)h * args.cap + zt.blk];
+  const int e1 = args.row_ptr[(int64_t)h * args.cap + zt.blk + 1];
+  const int row_base = (int)((int64_t)h * args.N);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(b_q, 1);
+    for (int s = 0; s < kDqKStages; ++s) {
+      tc::mbar_init(b_kfull(s), 1);
+      tc::mbar_init(b_kempty(s), 1);
+    }
+    for (int s = 0; s < kDqVStages; ++s) {
+      tc::mbar_init(b_vfull(s), 1);
+      tc::mbar_init(b_vempty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(b_sd(b), 1);
+      tc::mbar_init(b_ds(b), 128);
+    }
+    tc::mbar_init(b_drain, 1);
+    *abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto tS = [&](int b) { return tmem + 128u * (uint32_t)b; };
+  const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
+  const uint32_t limit = args.wait_limit;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmQ);
+      tc::prefetch_tmap(&tmK);
+      tc::prefetch_tmap(&tmV);
+      tc::prefetch_tmap(&tmO);
+      tc::mbar_expect_tx(b_q, 2 * kTcTileBytes);
+      tc::tma_load_2d(sQ, &tmQ, 0, row_base + zt.r0, b_q);
+      tc::tma_load_2d(sQ + kTcTileBytes / 2, &tmQ, 64, row_base + zt.r0, b_q);
+      tc::tma_load_2d(sO, &tmO, 0, row_base + zt.r0, b_q);
+      tc::tma_load_2d(sO + kTcTileBytes / 2, &tmO, 64, row_base + zt.r0, b_q);
+      KeyTiles kt;
+      kt.init(args.col, args.blocks, e0, e1);
+      int nk = 0, nv = 0;
+      for (; kt.valid(); kt.next()) {
+        const int ks = nk % kDqKStages, vs = nv % kDqVStages;
+        if (!tc::mbar_wait(b_kempty(ks), ((uint32_t)(nk / kDqKStages) & 1u) ^ 1u, abort, limit)) break;
+        tc::mbar_expect_tx(b_kfull(ks), kTcTileBytes);
+        tc::tma_load_2d(sK(ks), &tmK, 0, row_base + kt.row(), b_kfull(ks));
+        tc::tma_load_2d(sK(ks) + kTcTileBytes / 2, &tmK, 64, row_base + kt.row(), b_kfull(ks));
+        ++nk;
+        if (!tc::mbar_wait(b_vempty(vs), ((uint32_t)(nv / kDqVStages) & 1u) ^ 1u, abort, limit)) break;
+        tc::mbar_expect_tx(b_vfull(vs), kTcTileBytes);
+        tc::tma_load_2d(sV(vs), &tmV, 0, row_base + kt.row(), b_vfull(vs));
+        tc::tma_load_2d(sV(vs) + kTcTileBytes / 2, &tmV, 64, row_base + kt.row(), b_vfull(vs));
+        ++nv;
+      }
+      volatile int no_abort = 0;
+      tc::mbar_wait(b_q, 0, &no_abort, limit);
+      for (int k = max(0, nk - kDqKStages); k < nk; ++k)
+        tc::mbar_wait(b_kfull(k % kDqKStages), (uint32_t)(k / kDqKStages) & 1u, &no_abort, limit);
+      for (int k = max(0, nv - kDqVStages); k < nv; ++k)
+        tc::mbar_wait(b_vfull(k % kDqVStages), (uint32_t)(k / kDqVStages) & 1u, &no_abort, limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const int nsteps = count_key_tiles(args.col, args.blocks, e0, e1);
+      constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
+      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);    // B MN-major
+      bool ok = tc::mbar_wait(b_q, 0, abort, limit);
+      auto issue_s = [&](int n) -> bool {   // S_n = Q K_n^T
+        const int ks = n % kDqKStages;
+        if (!tc::mbar_wait(b_kfull(ks), (uint32_t)(n / kDqKStages) & 1u, abort, limit)) return false;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
+          tc::mma_ss(tS(n & 1), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK(ks) + off, 16, 1024), idNT,
+                     k > 0);
+        }
+        return true;
+      };
+      auto issue_dp = [&](int n) -> bool {   // dP_n = dO V_n^T
+        const int vs = n % kDqVStages;
+        if (!tc::mbar_wait(b_vfull(vs), (uint32_t)(n / kDqVStages) & 1u, abort, limit)) return false;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
+          tc::mma_ss(tdP, tc::sw128_desc(sO + off, 16, 1024), tc::sw128_desc(sV(vs) + off, 16, 1024), idNT,
+                     k > 0);
+        }
+        tc::mma_commit(b_vempty(vs));
+        tc::mma_commit(b_sd(n & 1));
+        return true;
+      };
+      if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
+      for (int n = 0; ok && n < nsteps; ++n) {
+        if (n + 1 < nsteps && !issue_s(n + 1)) break;
+        if (!tc::mbar_wait(b_ds(n & 1), (uint32_t)(n >> 1) & 1u, abort, limit)) break;
+        tc::tc_fence_after();
+        if (n + 1 < nsteps && !issue_dp(n + 1)) break;
+        const int ks = n % kDqKStages;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)   // dQ += dS_n K_n, 16 keys per step
+          tc::mma_ts(tdQ, tS(n & 1) + 8u * k, tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
+                     (n > 0 || k > 0) ? 1u : 0u);
+        tc::mma_commit(b_kempty(ks));
+      }
+      tc::mma_commit(b_drain);
+      volatile int no_abort = 0;
+      tc::mbar_wait(b_drain, 0, &no_abort, limit);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const float sl2 = args.scale_log2;
+    const int64_t grow = (int64_t)h * args.N + zt.r0 + row;
+    const bool vrow = row < zt.rows;
+    const float lse2 = vrow ? args.lse[grow] * kLog2e : INFINITY;   // padding rows: P = 0
+    const float dl = vrow ? args.delta[grow] : 0.f;
+    KeyTiles kt;
+    kt.init(args.col, args.blocks, e0, e1);
+    int n = 0;
+    bool ok = true;
+    for (; kt.valid(); kt.next(), ++n) {
+      const int b = n & 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_sd(b), (uint32_t)(n >> 1) & 1u, abort, limit))) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      const int kv = kt.keys();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], pv[32], pk[16];
+        tc::tmem_ld32(tS(b) + lane_off + 32u * c, sv);
+        tc::tmem_ld32(tdP + lane_off + 32u * c, pv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = 32 * c + 2 * e;
+          const float p0 = (c0 < kv) ? exp2f(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse2)) : 0.f;
+          const float p1 = (c0 + 1 < kv) ? exp2f(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse2)) : 0.f;
+          pk[e] = pack_bf16(p0 * (__uint_as_float(pv[2 * e]) - dl), p1 * (__uint_as_float(pv[2 * e + 1]) - dl));
+        }
+        tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
+      }
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(b_ds(b));
+    }
+    if (__all_sync(0xffffffffu, ok && !*abort) && vrow) {
+      bool have = n > 0;
+      if (have && !__all_sync(0xffffffffu, tc::mbar_wait(b_drain, 0, abort, limit))) have = false, ok = false;
+      if (ok) {
+        if (have) tc::tc_fence_after();
+        __nv_bfloat16 *out = args.dq + grow * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          if (have) {
+            tc::tmem_ld32(tdQ + lane_off + 32u * c, v);
+            tc::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+#pragma unroll
+          for (int v8 = 0; v8 < 4; ++v8) {
+            uint4 u;
+            uint32_t *up = &u.x;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              up[e] = pack_bf16(__uint_as_float(v[8 * v8 + 2 * e]) * args.scale,
+                                __uint_as_float(v[8 * v8 + 2 * e + 1]) * args.scale);
+            *reinterpret_cast<uint4 *>(out + 32 * c + 8 * v8) = u;
+          }
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ========================================================================= dK dV
+constexpr int kKvQStages = 2;
+// K, V, 2 x (Q, dO), dS^T tiles; barriers; alignment slack.
+constexpr int kKvSmemBytes = kTcTileBytes * (3 + 2 * kKvQStages) + 256 + 1024;
+
+__global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                             const __grid_constant__ CUtensorMap tmK,
+                                                             const __grid_constant__ CUtensorMap tmV,
+                                                             const __grid_constant__ CUtensorMap tmO,
+                                                             const TcBwdArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t *sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  const uint32_t sK = sbase, sV = sbase + kTcTileBytes, sdS = sbase + 2 * kTcTileBytes;
+  auto sQ = [&](int s) { return sbase + (uint32_t)(3 + 2 * s) * kTcTileBytes; };
+  auto sO = [&](int s) { return sbase + (uint32_t)(4 + 2 * s) * kTcTileBytes; };
+  const uint32_t sBar = sbase + (uint32_t)(3 + 2 * kKvQStages) * kTcTileBytes;
+  const uint32_t b_kv = sBar;
+  auto b_qfull = [&](int s) { return sBar + 8u * (1 + s); };    // Q_n and dO_n landed
+  auto b_qempty = [&](int s) { return sBar + 8u * (3 + s); };
+  const uint32_t b_st = sBar + 8u * 5;     // S^T_n and dP^T_n done
+  const uint32_t b_p = sBar + 8u * 6;      // P^T_n in TMEM, dS^T_n in smem (128 arrivals)
+  const uint32_t b_dsfree = sBar + 8u * 7; // dK_n finished reading dS^T
+  const uint32_t b_drain = sBar + 8u * 8;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 10);
+  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 10 + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  ZoneTile zt;
+  if (!zt.init(args.blocks, args.zone_blk_base, blockIdx.x >> 3, blockIdx.x & 7)) return;
+  const int e0 = args.col_ptr[(int64_t)h * args.cap + zt.blk];
+  const int e1 = args.col_ptr[(int64_t)h * args.cap + zt.blk + 1];
+  const int row_base = (int)((int64_t)h * args.N);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(b_kv, 1);
+    for (int s = 0; s < kKvQStages; ++s) {
+      tc::mbar_init(b_qfull(s), 1);
+      tc::mbar_init(b_qempty(s), 1);
+    }
+    tc::mbar_init(b_st, 1);
+    tc::mbar_init(b_p, 128);
+    tc::mbar_init(b_dsfree, 1);
+    tc::mbar_init(b_drain, 1);
+    *abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tdK = tmem, tdV = tmem + 128, tS = tmem + 256, tdP = tmem + 384;
+  const uint32_t limit = args.wait_limit;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmQ);
+      tc::prefetch_tmap(&tmK);
+      tc::prefetch_tmap(&tmV);
+      tc::prefetch_tmap(&tmO);
+      tc::mbar_expect_tx(b_kv, 2 * kTcTileBytes);
+      tc::tma_load_2d(sK, &tmK, 0, row_base + zt.r0, b_kv);
+      tc::tma_load_2d(sK + kTcTileBytes / 2, &tmK, 64, row_base + zt.r0, b_kv);
+      tc::tma_load_2d(sV, &tmV, 0, row_base + zt.r0, b_kv);
+      tc::tma_load_2d(sV + kTcTileBytes / 2, &tmV, 64, row_base + zt.r0, b_kv);
+      KeyTiles qt;   // query sub-tiles of the query blocks that selected this key block
+      qt.init(args.row_idx, args.blocks, e0, e1);
+      int nq = 0;
+      for (; qt.valid(); qt.next()) {
+        const int s = nq % kKvQStages;
+        if (!tc::mbar_wait(b_qempty(s), ((uint32_t)(nq / kKvQStages) & 1u) ^ 1u, abort, limit)) break;
+        tc::mbar_expect_tx(b_qfull(s), 2 * kTcTileBytes);
+        tc::tma_load_2d(sQ(s), &tmQ, 0, row_base + qt.row(), b_qfull(s));
+        tc::tma_load_2d(sQ(s) + kTcTileBytes / 2, &tmQ, 64, row_base + qt.row(), b_qfull(s));
+        tc::tma_load_2d(sO(s), &tmO, 0, row_base + qt.row(), b_qfull(s));
+        tc::tma_load_2d(sO(s) + kTcTileBytes / 2, &tmO, 64, row_base + qt.row(), b_qfull(s));
+        ++nq;
+      }
+      volatile int no_abort = 0;
+      tc::mbar_wait(b_kv, 0, &no_abort, limit);
+      for (int k = max(0, nq - kKvQStages); k < nq; ++k)
+        tc::mbar_wait(b_qfull(k % kKvQStages), (uint32_t)(k / kKvQStages) & 1u, &no_abort, limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const int nsteps = count_key_tiles(args.row_idx, args.blocks, e0, e1);
+      constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);
+      bool ok = tc::mbar_wait(b_kv, 0, abort, limit);
+      for (int n = 0; ok && n < nsteps; ++n) {
+        const int s = n % kKvQStages;
+        if (!tc::mbar_wait(b_qfull(s), (uint32_t)(n / kKvQStages) & 1u, abort, limit)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {   // S^T = K Q^T ; dP^T = V dO^T
+          const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
+          tc::mma_ss(tS, tc::sw128_desc(sK + off, 16, 1024), tc::sw128_desc(sQ(s) + off, 16, 1024), idNT, k > 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
+          tc::mma_ss(tdP, tc::sw128_desc(sV + off, 16, 1024), tc::sw128_desc(sO(s) + off, 16, 1024), idNT, k > 0);
+        }
+        tc::mma_commit(b_st);
+        if (!tc::mbar_wait(b_p, (uint32_t)n & 1u, abort, limit)) break;
+        tc::tc_fence_after();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)   // dV += P^T dO, 16 queries per step
+          tc::mma_ts(tdV, tS + 8u * k, tc::sw128_desc(sO(s) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
+                     (n > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {  // dK += dS^T Q
+          const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
+          tc::mma_ss(tdK, tc::sw128_desc(sdS + off, 16, 1024),
+                     tc::sw128_desc(sQ(s) + 2048u * k, kTcTileBytes / 2, 1024), idMN, (n > 0 || k > 0) ? 1u : 0u);
+        }
+        tc::mma_commit(b_dsfree);
+        tc::mma_commit(b_qempty(s));
+      }
+      tc::mma_commit(b_drain);
+      volatile int no_abort = 0;
+      tc::mbar_wait(b_drain, 0, &no_abort, limit);
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = 32 * q + lane;        // key row of the tile
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const float sl2 = args.scale_log2;
+    uint8_t *dsrow = sgen + (sdS - sbase) + row * 128;
+    KeyTiles qt;
+    qt.init(args.row_idx, args.blocks, e0, e1);
+    int n = 0;
+    bool ok = true;
+    for (; qt.valid(); qt.next(), ++n) {
+      const int qv = qt.keys();   // valid queries in this tile
+      // per-column LSE and D of the query tile: the same addresses for every
+      // thread, served as broadcasts from L1
+      const float *lse_t = args.lse + (int64_t)h * args.N + qt.row();
+      const float *dl_t = args.delta + (int64_t)h * args.N + qt.row();
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_st, (uint32_t)n & 1u, abort, limit))) {
+        ok = false;
+        break;
+      }
+      if (n > 0 && !__all_sync(0xffffffffu, tc::mbar_wait(b_dsfree, (uint32_t)(n - 1) & 1u, abort, limit))) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], pv[32], pk[16], dk[16];
+        tc::tmem_ld32(tS + lane_off + 32u * c, sv);
+        tc::tmem_ld32(tdP + lane_off + 32u * c, pv);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = 32 * c + 2 * e;
+          const bool v0 = c0 < qv, v1 = c0 + 1 < qv;   // padding columns: P = 0
+          const float l0 = v0 ? __ldg(lse_t + c0) * kLog2e : INFINITY;
+          const float l1 = v1 ? __ldg(lse_t + c0 + 1) * kLog2e : INFINITY;
+          const float d0 = v0 ? __ldg(dl_t + c0) : 0.f, d1 = v1 ? __ldg(dl_t + c0 + 1) : 0.f;
+          const float p0 = exp2f(fmaf(__uint_as_float(sv[2 * e]), sl2, -l0));
+          const float p1 = exp2f(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l1));
+          pk[e] = pack_bf16(p0, p1);
+          dk[e] = pack_bf16(p0 * (__uint_as_float(pv[2 * e]) - d0), p1 * (__uint_as_float(pv[2 * e + 1]) - d1));
+        }
+        tc::tmem_st16(tS + lane_off + 16u * c, pk);
+        // dS^T row into the 128-byte-swizzled K-major tile: columns 32c..32c+31
+        // are 16-byte chunks (c&1)*4+u of the 64-column half c>>1
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int chunk = ((c & 1) * 4 + u) ^ (row & 7);
+          *reinterpret_cast<uint4 *>(dsrow + (c >> 1) * (kTcTileBytes / 2) + chunk * 16) =
+              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+      }
+      tc::tmem_st_wait();
+      fence_proxy_async_smem();
+      tc::tc_fence_before();
+      tc::mbar_arrive(b_p);
+    }
+    if (__all_sync(0xffffffffu, ok && !*abort) && row < zt.rows) {
+      bool have = n > 0;
+      if (have && !__all_sync(0xffffffffu, tc::mbar_wait(b_drain, 0, abort, limit))) have = false, ok = false;
+      if (ok) {
+        if (have) tc::tc_fence_after();
+        const int64_t grow = (int64_t)h * args.N + zt.r0 + row;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          __nv_bfloat16 *out = (which ? args.dv : args.dk) + grow * 128;
+          const float mul = which ? 1.f : args.scale;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            if (have) {
+              tc::tmem_ld32((which ? tdV : tdK) + lane_off + 32u * c, v);
+              tc::tmem_ld_wait();
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = 0u;
+            }
+#pragma unroll
+            for (int v8 = 0; v8 < 4; ++v8) {
+              uint4 w;
+              uint32_t *wp = &w.x;
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                wp[e] = pack_bf16(__uint_as_float(v[8 * v8 + 2 * e]) * mul, __uint_as_float(v[8 * v8 + 2 * e + 1]) * mul);
+              *reinterpret_cast<uint4 *>(out + 32 * c + 8 * v8) = w;
+            }
+          }
+        }
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace prism

@@ -8,7 +8,7 @@
 #include <string>
 
 #include "attn_mma_bwd.cuh"
-#include "attn_tc_fwd.cuh"
+#include "attn_tc_bwd.cuh"
 #include "indicator.cuh"
 #include "permute.cuh"
 #include "select.cuh"
@@ -491,7 +491,35 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
   auto Q = static_cast<const __nv_bfloat16 *>(q), K = static_cast<const __nv_bfloat16 *>(k),
        Vv = static_cast<const __nv_bfloat16 *>(v);
   const float scale = eff_scale(p);
-  if (d.D == 128)
+  if (d.D == 128 && g_attn_backend == 0) {
+    CUtensorMap tq, tk, tv, to;
+    const uint64_t rows = (uint64_t)d.heads * d.N;
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
+        !make_tile_map(&to, dout, rows))
+      return fail(PRISM_ECUDA, "cuTensorMapEncodeTiled failed");
+    TcBwdArgs a;
+    a.blocks = blocks;
+    a.zone_blk_base = zone_blk_base;
+    a.row_ptr = row_ptr;
+    a.col = col;
+    a.col_ptr = col_ptr;
+    a.row_idx = row_idx;
+    a.lse = lse;
+    a.delta = delta;
+    a.N = d.N;
+    a.cap = d.cap;
+    a.scale = scale;
+    a.scale_log2 = scale * kLog2e;
+    a.dq = static_cast<__nv_bfloat16 *>(dq);
+    a.dk = static_cast<__nv_bfloat16 *>(dk);
+    a.dv = static_cast<__nv_bfloat16 *>(dv);
+    a.wait_limit = g_wait_limit ? g_wait_limit : kDefaultWaitLimit;
+    cudaFuncSetAttribute(bsa_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemBytes);
+    cudaFuncSetAttribute(bsa_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmemBytes);
+    dim3 tgrid((unsigned)(d.Z * 8), d.heads);
+    PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, 192, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
+    PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, 192, kDqSmemBytes, st>>>(tq, tk, tv, to, a));
+  } else if (d.D == 128)
     launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
                          row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
                          static_cast<__nv_bfloat16 *>(dv));
