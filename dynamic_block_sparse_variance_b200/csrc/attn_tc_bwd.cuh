@@ -240,8 +240,8 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c0 = 32 * c + 2 * e;
-          const float p0 = (c0 < kv) ? exp2f(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse2)) : 0.f;
-          const float p1 = (c0 + 1 < kv) ? exp2f(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse2)) : 0.f;
+          const float p0 = (c0 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse2)) : 0.f;
+          const float p1 = (c0 + 1 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse2)) : 0.f;
           pk[e] = pack_bf16(p0 * (__uint_as_float(pv[2 * e]) - dl), p1 * (__uint_as_float(pv[2 * e + 1]) - dl));
         }
         tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
@@ -454,8 +454,8 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
           const float l0 = v0 ? __ldg(lse_t + c0) * kLog2e : INFINITY;
           const float l1 = v1 ? __ldg(lse_t + c0 + 1) * kLog2e : INFINITY;
           const float d0 = v0 ? __ldg(dl_t + c0) : 0.f, d1 = v1 ? __ldg(dl_t + c0 + 1) : 0.f;
-          const float p0 = exp2f(fmaf(__uint_as_float(sv[2 * e]), sl2, -l0));
-          const float p1 = exp2f(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l1));
+          const float p0 = tc::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -l0));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l1));
           pk[e] = pack_bf16(p0, p1);
           dk[e] = pack_bf16(p0 * (__uint_as_float(pv[2 * e]) - d0), p1 * (__uint_as_float(pv[2 * e + 1]) - d1));
         }

@@ -247,19 +247,25 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
       for (int c = 0; c < 4; ++c) tc::tmem_ld32(tS(b) + lane_off + 32u * c, raw[c]);
       tc::tmem_ld_wait();
       const int kv = kt.keys();
-      float mx = -INFINITY;
+      if (kv < 128) {   // a 64-key block: the upper half of the tile is padding
+#pragma unroll
+        for (int c = 2; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) raw[c][e] = __float_as_uint(-INFINITY);
+      }
+      // row max with eight independent chains
+      float m8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float v = (32 * c + e < kv) ? __uint_as_float(raw[c][e]) : -INFINITY;
-          raw[c][e] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
+        for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= sl2;
       // lazy rescaling: only rows whose max grew by more than 2^8 move m_run
       const bool grow = mx > m_run + 8.f;
-      const float alpha = grow ? exp2f(m_run - mx) : 1.f;
+      const float alpha = grow ? tc::ex2(m_run - mx) : 1.f;
       if (grow) {
         l_run *= alpha;
         m_run = mx;
@@ -282,20 +288,22 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
           tc::tmem_st32(tO + lane_off + 32u * c, ov);
         }
       }
-      float rs = 0.f;
+      float r8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2f(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
-          const float p1 = exp2f(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
-          rs += p0 + p1;
+          const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
+          r8[e & 7] += p0 + p1;
           pk[e] = pack_bf16(p0, p1);
         }
         tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
       }
-      l_run += rs;
+      l_run += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tmem_st_wait();
       tc::tc_fence_before();
       if (!(args.debug_stall && n == 0)) tc::mbar_arrive(b_pfull(b));
