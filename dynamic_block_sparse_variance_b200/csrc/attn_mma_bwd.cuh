@@ -19,7 +19,8 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16 *__restrict__ o,
                                                         const __nv_bfloat16 *__restrict__ o_res,
                                                         const __nv_bfloat16 *__restrict__ dout,
-                                                        int64_t rows, float *__restrict__ delta) {
+                                                        const float *__restrict__ lse, int64_t rows,
+                                                        float *__restrict__ delta, float *__restrict__ lse2) {
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
@@ -39,7 +40,10 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16 *__r
     s += o0 * bf16_lo(ub) + o1 * bf16_hi(ub);
   }
   s = warp_sum(s);
-  if (lane == 0) delta[r] = s;
+  if (lane == 0) {
+    delta[r] = s;
+    lse2[r] = lse[r] * 1.4426950408889634f;   // LSE in log2 units for the key-side kernel
+  }
 }
 
 // ---- CSR -> CSC per head -------------------------------------------------

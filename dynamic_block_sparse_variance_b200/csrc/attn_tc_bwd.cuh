@@ -32,6 +32,8 @@ struct TcBwdArgs {
   const int32_t *row_idx;
   const float *lse;
   const float *delta;
+  const float *lse2_pad;    // dkdv: LSE*log2e and D, padded by 128 entries
+  const float *delta_pad;
   int64_t N, cap;
   float scale_log2, scale;
   __nv_bfloat16 *dq, *dk, *dv;
@@ -290,8 +292,10 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
 
 // ========================================================================= dK dV
 constexpr int kKvQStages = 2;
-// K, V, 2 x (Q, dO), dS^T tiles; barriers; alignment slack.
-constexpr int kKvSmemBytes = kTcTileBytes * (3 + 2 * kKvQStages) + 256 + 1024;
+// K, V, dS^T, 2 x (Q, dO) tiles; 2 x (LSE*log2e, D) rows of 128 floats;
+// barriers.  The dynamic shared window starts 1024-byte aligned (no static
+// shared memory in these kernels); the kernel checks it.
+constexpr int kKvSmemBytes = kTcTileBytes * (3 + 2 * kKvQStages) + 2 * 1024 + 256;
 
 __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                              const __grid_constant__ CUtensorMap tmK,
@@ -301,10 +305,16 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t *sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  if (sbase != smem_u32(smem_raw)) {   // the layout has no alignment slack
+    if (threadIdx.x == 0) set_status(PRISM_EBOUNDS);
+    return;
+  }
   const uint32_t sK = sbase, sV = sbase + kTcTileBytes, sdS = sbase + 2 * kTcTileBytes;
   auto sQ = [&](int s) { return sbase + (uint32_t)(3 + 2 * s) * kTcTileBytes; };
   auto sO = [&](int s) { return sbase + (uint32_t)(4 + 2 * s) * kTcTileBytes; };
-  const uint32_t sBar = sbase + (uint32_t)(3 + 2 * kKvQStages) * kTcTileBytes;
+  const uint32_t sStat0 = sbase + (uint32_t)(3 + 2 * kKvQStages) * kTcTileBytes;   // [2][256] floats
+  auto sStat = [&](int s) { return sStat0 + 1024u * (uint32_t)s; };
+  const uint32_t sBar = sStat0 + 2048;
   const uint32_t b_kv = sBar;
   auto b_qfull = [&](int s) { return sBar + 8u * (1 + s); };    // Q_n and dO_n landed
   auto b_qempty = [&](int s) { return sBar + 8u * (3 + s); };
@@ -364,7 +374,9 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
       for (; qt.valid(); qt.next()) {
         const int s = nq % kKvQStages;
         if (!tc::mbar_wait(b_qempty(s), ((uint32_t)(nq / kKvQStages) & 1u) ^ 1u, abort, limit)) break;
-        tc::mbar_expect_tx(b_qfull(s), 2 * kTcTileBytes);
+        tc::mbar_expect_tx(b_qfull(s), 2 * kTcTileBytes + 1024);
+        tc::bulk_load(sStat(s), args.lse2_pad + row_base + qt.row(), 512, b_qfull(s));
+        tc::bulk_load(sStat(s) + 512, args.delta_pad + row_base + qt.row(), 512, b_qfull(s));
         tc::tma_load_2d(sQ(s), &tmQ, 0, row_base + qt.row(), b_qfull(s));
         tc::tma_load_2d(sQ(s) + kTcTileBytes / 2, &tmQ, 64, row_base + qt.row(), b_qfull(s));
         tc::tma_load_2d(sO(s), &tmO, 0, row_base + qt.row(), b_qfull(s));
@@ -428,10 +440,14 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
     bool ok = true;
     for (; qt.valid(); qt.next(), ++n) {
       const int qv = qt.keys();   // valid queries in this tile
-      // per-column LSE and D of the query tile: the same addresses for every
-      // thread, served as broadcasts from L1
-      const float *lse_t = args.lse + (int64_t)h * args.N + qt.row();
-      const float *dl_t = args.delta + (int64_t)h * args.N + qt.row();
+      const int s = n % kKvQStages;
+      // this tile's LSE*log2e and D rows, bulk-copied by the producer with Q and dO
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_qfull(s), (uint32_t)(n / kKvQStages) & 1u, abort, limit))) {
+        ok = false;
+        break;
+      }
+      const float *st_l = reinterpret_cast<const float *>(sgen + (sStat(s) - sbase));
+      const float *st_d = st_l + 128;
       if (!__all_sync(0xffffffffu, tc::mbar_wait(b_st, (uint32_t)n & 1u, abort, limit))) {
         ok = false;
         break;
@@ -451,9 +467,8 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
         for (int e = 0; e < 16; ++e) {
           const int c0 = 32 * c + 2 * e;
           const bool v0 = c0 < qv, v1 = c0 + 1 < qv;   // padding columns: P = 0
-          const float l0 = v0 ? __ldg(lse_t + c0) * kLog2e : INFINITY;
-          const float l1 = v1 ? __ldg(lse_t + c0 + 1) * kLog2e : INFINITY;
-          const float d0 = v0 ? __ldg(dl_t + c0) : 0.f, d1 = v1 ? __ldg(dl_t + c0 + 1) : 0.f;
+          const float l0 = v0 ? st_l[c0] : INFINITY, l1 = v1 ? st_l[c0 + 1] : INFINITY;
+          const float d0 = v0 ? st_d[c0] : 0.f, d1 = v1 ? st_d[c0 + 1] : 0.f;
           const float p0 = tc::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -l0));
           const float p1 = tc::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l1));
           pk[e] = pack_bf16(p0, p1);

@@ -127,13 +127,15 @@ struct SelectWs {
   }
 };
 struct BwdWs {
-  size_t delta, ccnt, col_ptr, fill, part, tot, row_idx, total;
+  size_t delta, lse2, ccnt, col_ptr, fill, part, tot, row_idx, total;
   int64_t R, nchunk;
   BwdWs(const Dims &d, int64_t col_capacity) {
     R = (int64_t)d.heads * d.cap;
     nchunk = (R + kScanChunk - 1) / kScanChunk;
+    // D and LSE*log2e, each padded by 128 entries for whole-tile bulk copies
     delta = 0;
-    ccnt = align256((size_t)d.heads * d.N * 4);
+    lse2 = align256(((size_t)d.heads * d.N + 128) * 4);
+    ccnt = lse2 + align256(((size_t)d.heads * d.N + 128) * 4);
     col_ptr = ccnt + align256(R * 4);
     fill = col_ptr + align256((R + 1) * 4);
     part = fill + align256(R * 4);
@@ -462,6 +464,7 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
   cudaStream_t st = as_stream(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   float *delta = reinterpret_cast<float *>(ws + w.delta);
+  float *lse2 = reinterpret_cast<float *>(ws + w.lse2);
   int32_t *ccnt = reinterpret_cast<int32_t *>(ws + w.ccnt);
   int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + w.col_ptr);
   int32_t *fill = reinterpret_cast<int32_t *>(ws + w.fill);
@@ -472,9 +475,11 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
   if (o_res && !aligned16(o_res)) return fail(PRISM_EINVAL, "bwd: o_res must be 16-byte aligned");
   const int64_t rows = (int64_t)d.heads * d.N;
   if (d.D == 128)
-    PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, rows, delta));
+    PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, lse, rows, delta, lse2));
   else
-    PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<64><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, rows, delta));
+    PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<64><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, lse, rows, delta, lse2));
+  cudaMemsetAsync(delta + rows, 0, 128 * 4, st);
+  cudaMemsetAsync(lse2 + rows, 0, 128 * 4, st);
   cudaMemsetAsync(ccnt, 0, w.R * 4, st);
   cudaMemsetAsync(fill, 0, w.R * 4, st);
   dim3 rgrid((unsigned)d.cap, d.heads);
@@ -506,6 +511,8 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
     a.row_idx = row_idx;
     a.lse = lse;
     a.delta = delta;
+    a.lse2_pad = lse2;
+    a.delta_pad = delta;
     a.N = d.N;
     a.cap = d.cap;
     a.scale = scale;
