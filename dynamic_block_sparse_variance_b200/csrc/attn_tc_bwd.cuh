@@ -16,7 +16,15 @@
 //   and dS^T (written to 128-byte-swizzled shared memory, the A operand of
 //   dK += dS^T Q_n).  TMEM: dK | dV | S^T | dP^T.
 //
-// Roles, bounded waits and the abort path follow the forward kernel.
+// Roles, bounded waits and the abort path follow the forward kernel, with
+// eight elementwise warps instead of four: warps w and w+4 share a TMEM lane
+// quadrant and take the lower and upper 64 columns of each row (the backward
+// needs no row reduction).  A half writes its bf16 results into the first 32
+// columns of its own 64-column range, so operand k-step k (16 elements) sits
+// at column 8k + (k >= 4 ? 32 : 0).
+
+constexpr int kBwdThreads = 320;   // producer, MMA, 8 elementwise warps
+__device__ __forceinline__ uint32_t half_col(int k) { return 8u * (uint32_t)k + (k >= 4 ? 32u : 0u); }
 #pragma once
 
 #include "attn_tc_fwd.cuh"
@@ -68,7 +76,7 @@ struct ZoneTile {
 constexpr int kDqKStages = 3, kDqVStages = 2;
 constexpr int kDqSmemBytes = kTcTileBytes * (2 + kDqKStages + kDqVStages) + 256 + 1024;
 
-__global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                            const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const __grid_constant__ CUtensorMap tmO,
@@ -111,7 +119,7 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(b_sd(b), 1);
-      tc::mbar_init(b_ds(b), 128);
+      tc::mbar_init(b_ds(b), 256);
     }
     tc::mbar_init(b_drain, 1);
     *abort = 0;
@@ -204,7 +212,7 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
         const int ks = n % kDqKStages;
 #pragma unroll
         for (int k = 0; k < 8; ++k)   // dQ += dS_n K_n, 16 keys per step
-          tc::mma_ts(tdQ, tS(n & 1) + 8u * k, tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
+          tc::mma_ts(tdQ, tS(n & 1) + half_col(k), tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
                      (n > 0 || k > 0) ? 1u : 0u);
         tc::mma_commit(b_kempty(ks));
       }
@@ -214,6 +222,7 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
     }
   } else {
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;        // columns [64*half, 64*half + 64)
     const int row = 32 * q + lane;
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const float sl2 = args.scale_log2;
@@ -233,20 +242,24 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
       }
       tc::tc_fence_after();
       const int kv = kt.keys();
+      uint32_t sv[2][32], pv[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32], pv[32], pk[16];
-        tc::tmem_ld32(tS(b) + lane_off + 32u * c, sv);
-        tc::tmem_ld32(tdP + lane_off + 32u * c, pv);
-        tc::tmem_ld_wait();
+      for (int cc = 0; cc < 2; ++cc) {
+        tc::tmem_ld32(tS(b) + lane_off + 64u * half + 32u * cc, sv[cc]);
+        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, pv[cc]);
+      }
+      tc::tmem_ld_wait();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * c + 2 * e;
-          const float p0 = (c0 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -lse2)) : 0.f;
-          const float p1 = (c0 + 1 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -lse2)) : 0.f;
-          pk[e] = pack_bf16(p0 * (__uint_as_float(pv[2 * e]) - dl), p1 * (__uint_as_float(pv[2 * e + 1]) - dl));
+          const int c0 = 64 * half + 32 * cc + 2 * e;
+          const float p0 = (c0 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e]), sl2, -lse2)) : 0.f;
+          const float p1 = (c0 + 1 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e + 1]), sl2, -lse2)) : 0.f;
+          pk[e] = pack_bf16(p0 * (__uint_as_float(pv[cc][2 * e]) - dl), p1 * (__uint_as_float(pv[cc][2 * e + 1]) - dl));
         }
-        tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
+        tc::tmem_st16(tS(b) + lane_off + 64u * half + 16u * cc, pk);
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
@@ -257,12 +270,12 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
       if (have && !__all_sync(0xffffffffu, tc::mbar_wait(b_drain, 0, abort, limit))) have = false, ok = false;
       if (ok) {
         if (have) tc::tc_fence_after();
-        __nv_bfloat16 *out = args.dq + grow * 128;
+        __nv_bfloat16 *out = args.dq + grow * 128 + 64 * half;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t v[32];
           if (have) {
-            tc::tmem_ld32(tdQ + lane_off + 32u * c, v);
+            tc::tmem_ld32(tdQ + lane_off + 64u * half + 32u * cc, v);
             tc::tmem_ld_wait();
           } else {
 #pragma unroll
@@ -276,7 +289,7 @@ __global__ void __launch_bounds__(192, 1) bsa_dq_tc_kernel(const __grid_constant
             for (int e = 0; e < 4; ++e)
               up[e] = pack_bf16(__uint_as_float(v[8 * v8 + 2 * e]) * args.scale,
                                 __uint_as_float(v[8 * v8 + 2 * e + 1]) * args.scale);
-            *reinterpret_cast<uint4 *>(out + 32 * c + 8 * v8) = u;
+            *reinterpret_cast<uint4 *>(out + 32 * cc + 8 * v8) = u;
           }
         }
       }
@@ -297,7 +310,7 @@ constexpr int kKvQStages = 2;
 // shared memory in these kernels); the kernel checks it.
 constexpr int kKvSmemBytes = kTcTileBytes * (3 + 2 * kKvQStages) + 2 * 1024 + 256;
 
-__global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                              const __grid_constant__ CUtensorMap tmK,
                                                              const __grid_constant__ CUtensorMap tmV,
                                                              const __grid_constant__ CUtensorMap tmO,
@@ -340,7 +353,7 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
       tc::mbar_init(b_qempty(s), 1);
     }
     tc::mbar_init(b_st, 1);
-    tc::mbar_init(b_p, 128);
+    tc::mbar_init(b_p, 256);
     tc::mbar_init(b_dsfree, 1);
     tc::mbar_init(b_drain, 1);
     *abort = 0;
@@ -413,7 +426,7 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
         tc::tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k)   // dV += P^T dO, 16 queries per step
-          tc::mma_ts(tdV, tS + 8u * k, tc::sw128_desc(sO(s) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
+          tc::mma_ts(tdV, tS + half_col(k), tc::sw128_desc(sO(s) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
                      (n > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {  // dK += dS^T Q
@@ -430,10 +443,11 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
     }
   } else {
     const int q = warp & 3;
-    const int row = 32 * q + lane;        // key row of the tile
+    const int half = (warp - 2) >> 2;        // query columns [64*half, 64*half + 64)
+    const int row = 32 * q + lane;           // key row of the tile
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const float sl2 = args.scale_log2;
-    uint8_t *dsrow = sgen + (sdS - sbase) + row * 128;
+    uint8_t *dsrow = sgen + (sdS - sbase) + row * 128 + half * (kTcTileBytes / 2);
     KeyTiles qt;
     qt.init(args.row_idx, args.blocks, e0, e1);
     int n = 0;
@@ -446,8 +460,8 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
         ok = false;
         break;
       }
-      const float *st_l = reinterpret_cast<const float *>(sgen + (sStat(s) - sbase));
-      const float *st_d = st_l + 128;
+      const float4 *st_l = reinterpret_cast<const float4 *>(sgen + (sStat(s) - sbase)) + 16 * half;
+      const float4 *st_d = st_l + 32;
       if (!__all_sync(0xffffffffu, tc::mbar_wait(b_st, (uint32_t)n & 1u, abort, limit))) {
         ok = false;
         break;
@@ -457,30 +471,46 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
         break;
       }
       tc::tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t sv[32], pv[32], pk[16], dk[16];
-        tc::tmem_ld32(tS + lane_off + 32u * c, sv);
-        tc::tmem_ld32(tdP + lane_off + 32u * c, pv);
-        tc::tmem_ld_wait();
+      uint32_t sv[2][32], pv[2][32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 32 * c + 2 * e;
-          const bool v0 = c0 < qv, v1 = c0 + 1 < qv;   // padding columns: P = 0
-          const float l0 = v0 ? st_l[c0] : INFINITY, l1 = v1 ? st_l[c0 + 1] : INFINITY;
-          const float d0 = v0 ? st_d[c0] : 0.f, d1 = v1 ? st_d[c0 + 1] : 0.f;
-          const float p0 = tc::ex2(fmaf(__uint_as_float(sv[2 * e]), sl2, -l0));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(sv[2 * e + 1]), sl2, -l1));
-          pk[e] = pack_bf16(p0, p1);
-          dk[e] = pack_bf16(p0 * (__uint_as_float(pv[2 * e]) - d0), p1 * (__uint_as_float(pv[2 * e + 1]) - d1));
+      for (int cc = 0; cc < 2; ++cc) {
+        tc::tmem_ld32(tS + lane_off + 64u * half + 32u * cc, sv[cc]);
+        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, pv[cc]);
+      }
+      tc::tmem_ld_wait();
+      const bool full = qv >= 64 * half + 64;   // no padding columns in this half
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {   // four query columns at a time
+          float4 L = st_l[8 * cc + g], Dv = st_d[8 * cc + g];
+          if (!full) {
+            const int c0 = 64 * half + 32 * cc + 4 * g;
+            if (c0 + 0 >= qv) { L.x = INFINITY; Dv.x = 0.f; }
+            if (c0 + 1 >= qv) { L.y = INFINITY; Dv.y = 0.f; }
+            if (c0 + 2 >= qv) { L.z = INFINITY; Dv.z = 0.f; }
+            if (c0 + 3 >= qv) { L.w = INFINITY; Dv.w = 0.f; }
+          }
+          const float p0 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 0]), sl2, -L.x));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 1]), sl2, -L.y));
+          const float p2 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 2]), sl2, -L.z));
+          const float p3 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 3]), sl2, -L.w));
+          pk[2 * g] = pack_bf16(p0, p1);
+          pk[2 * g + 1] = pack_bf16(p2, p3);
+          dk[2 * g] = pack_bf16(p0 * (__uint_as_float(pv[cc][4 * g + 0]) - Dv.x),
+                                p1 * (__uint_as_float(pv[cc][4 * g + 1]) - Dv.y));
+          dk[2 * g + 1] = pack_bf16(p2 * (__uint_as_float(pv[cc][4 * g + 2]) - Dv.z),
+                                    p3 * (__uint_as_float(pv[cc][4 * g + 3]) - Dv.w));
         }
-        tc::tmem_st16(tS + lane_off + 16u * c, pk);
-        // dS^T row into the 128-byte-swizzled K-major tile: columns 32c..32c+31
-        // are 16-byte chunks (c&1)*4+u of the 64-column half c>>1
+        tc::tmem_st16(tS + lane_off + 64u * half + 16u * cc, pk);
+        // dS^T row into the 128-byte-swizzled K-major tile: this half's 64
+        // columns are the half-tile `half`; columns 32cc..32cc+31 of it are
+        // 16-byte chunks 4cc..4cc+3
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int chunk = ((c & 1) * 4 + u) ^ (row & 7);
-          *reinterpret_cast<uint4 *>(dsrow + (c >> 1) * (kTcTileBytes / 2) + chunk * 16) =
+          const int chunk = (4 * cc + u) ^ (row & 7);
+          *reinterpret_cast<uint4 *>(dsrow + chunk * 16) =
               make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
         }
       }
@@ -497,13 +527,13 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
         const int64_t grow = (int64_t)h * args.N + zt.r0 + row;
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
-          __nv_bfloat16 *out = (which ? args.dv : args.dk) + grow * 128;
+          __nv_bfloat16 *out = (which ? args.dv : args.dk) + grow * 128 + 64 * half;
           const float mul = which ? 1.f : args.scale;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int cc = 0; cc < 2; ++cc) {
             uint32_t v[32];
             if (have) {
-              tc::tmem_ld32((which ? tdV : tdK) + lane_off + 32u * c, v);
+              tc::tmem_ld32((which ? tdV : tdK) + lane_off + 64u * half + 32u * cc, v);
               tc::tmem_ld_wait();
             } else {
 #pragma unroll
@@ -516,7 +546,7 @@ __global__ void __launch_bounds__(192, 1) bsa_dkdv_tc_kernel(const __grid_consta
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 wp[e] = pack_bf16(__uint_as_float(v[8 * v8 + 2 * e]) * mul, __uint_as_float(v[8 * v8 + 2 * e + 1]) * mul);
-              *reinterpret_cast<uint4 *>(out + 32 * c + 8 * v8) = w;
+              *reinterpret_cast<uint4 *>(out + 32 * cc + 8 * v8) = w;
             }
           }
         }

@@ -524,8 +524,8 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
     cudaFuncSetAttribute(bsa_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemBytes);
     cudaFuncSetAttribute(bsa_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmemBytes);
     dim3 tgrid((unsigned)(d.Z * 8), d.heads);
-    PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, 192, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
-    PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, 192, kDqSmemBytes, st>>>(tq, tk, tv, to, a));
+    PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, kBwdThreads, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
+    PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, kBwdThreads, kDqSmemBytes, st>>>(tq, tk, tv, to, a));
   } else if (d.D == 128)
     launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
                          row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
