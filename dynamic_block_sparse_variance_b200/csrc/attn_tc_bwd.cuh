@@ -93,8 +93,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   auto b_kempty = [&](int s) { return sBar + 8u * (4 + s); };   // 3
   auto b_vfull = [&](int s) { return sBar + 8u * (7 + s); };    // 2
   auto b_vempty = [&](int s) { return sBar + 8u * (9 + s); };   // 2
-  auto b_sd = [&](int b) { return sBar + 8u * (11 + b); };      // S_n and dP_n done
-  auto b_ds = [&](int b) { return sBar + 8u * (13 + b); };      // dS_n written (128 arrivals)
+  auto b_sd = [&](int hf) { return sBar + 8u * (11 + hf); };     // S and dP of key half hf done
+  auto b_ds = [&](int hf) { return sBar + 8u * (13 + hf); };     // dS of key half hf written (128 arrivals)
   const uint32_t b_drain = sBar + 8u * 15;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 16);
   volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 16 + 4);
@@ -117,9 +117,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       tc::mbar_init(b_vfull(s), 1);
       tc::mbar_init(b_vempty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(b_sd(b), 1);
-      tc::mbar_init(b_ds(b), 256);
+    for (int hf = 0; hf < 2; ++hf) {
+      tc::mbar_init(b_sd(hf), 1);
+      tc::mbar_init(b_ds(hf), 128);
     }
     tc::mbar_init(b_drain, 1);
     *abort = 0;
@@ -133,8 +133,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  auto tS = [&](int b) { return tmem + 128u * (uint32_t)b; };
-  const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
+  // dQ | S half A | S half B | dP half A | dP half B  (halves: keys 0-63, 64-127)
+  const uint32_t tdQ = tmem;
+  auto tS = [&](int hf) { return tmem + 128u + 64u * (uint32_t)hf; };
+  auto tP = [&](int hf) { return tmem + 256u + 64u * (uint32_t)hf; };
   const uint32_t limit = args.wait_limit;
 
   if (warp == 0) {
@@ -174,47 +176,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   } else if (warp == 1) {
     if (lane == 0) {
       const int nsteps = count_key_tiles(args.col, args.blocks, e0, e1);
-      constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
-      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);    // B MN-major
+      constexpr uint32_t idH = tc::idesc_bf16(128, 64, false, false);    // S, dP halves: N = 64 keys
+      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);   // dQ: B MN-major
       bool ok = tc::mbar_wait(b_q, 0, abort, limit);
-      auto issue_s = [&](int n) -> bool {   // S_n = Q K_n^T
-        const int ks = n % kDqKStages;
-        if (!tc::mbar_wait(b_kfull(ks), (uint32_t)(n / kDqKStages) & 1u, abort, limit)) return false;
-        tc::tc_fence_after();
+      // S_hf = Q K_hf^T and dP_hf = dO V_hf^T for key half hf of tile n
+      auto issue_sd = [&](int n, int hf) {
+        const int ks = n % kDqKStages, vs = n % kDqVStages;
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tS(n & 1), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK(ks) + off, 16, 1024), idNT,
-                     k > 0);
+          tc::mma_ss(tS(hf), tc::sw128_desc(sQ + off, 16, 1024),
+                     tc::sw128_desc(sK(ks) + 8192u * hf + off, 16, 1024), idH, k > 0);
         }
-        return true;
-      };
-      auto issue_dp = [&](int n) -> bool {   // dP_n = dO V_n^T
-        const int vs = n % kDqVStages;
-        if (!tc::mbar_wait(b_vfull(vs), (uint32_t)(n / kDqVStages) & 1u, abort, limit)) return false;
-        tc::tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tdP, tc::sw128_desc(sO + off, 16, 1024), tc::sw128_desc(sV(vs) + off, 16, 1024), idNT,
-                     k > 0);
+          tc::mma_ss(tP(hf), tc::sw128_desc(sO + off, 16, 1024),
+                     tc::sw128_desc(sV(vs) + 8192u * hf + off, 16, 1024), idH, k > 0);
         }
-        tc::mma_commit(b_vempty(vs));
-        tc::mma_commit(b_sd(n & 1));
-        return true;
+        tc::mma_commit(b_sd(hf));
       };
-      if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
+      auto wait_kv = [&](int n) -> bool {
+        return tc::mbar_wait(b_kfull(n % kDqKStages), (uint32_t)(n / kDqKStages) & 1u, abort, limit) &&
+               tc::mbar_wait(b_vfull(n % kDqVStages), (uint32_t)(n / kDqVStages) & 1u, abort, limit);
+      };
+      if (ok && nsteps > 0) {
+        ok = wait_kv(0);
+        if (ok) {
+          tc::tc_fence_after();
+          issue_sd(0, 0);
+          issue_sd(0, 1);
+        }
+      }
       for (int n = 0; ok && n < nsteps; ++n) {
-        if (n + 1 < nsteps && !issue_s(n + 1)) break;
-        if (!tc::mbar_wait(b_ds(n & 1), (uint32_t)(n >> 1) & 1u, abort, limit)) break;
-        tc::tc_fence_after();
-        if (n + 1 < nsteps && !issue_dp(n + 1)) break;
-        const int ks = n % kDqKStages;
+        const int ks = n % kDqKStages, vs = n % kDqVStages;
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          if (!tc::mbar_wait(b_ds(hf), (uint32_t)n & 1u, abort, limit)) { ok = false; break; }
+          tc::tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 8; ++k)   // dQ += dS_n K_n, 16 keys per step
-          tc::mma_ts(tdQ, tS(n & 1) + half_col(k), tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
-                     (n > 0 || k > 0) ? 1u : 0u);
-        tc::mma_commit(b_kempty(ks));
+          for (int k = 0; k < 4; ++k)   // dQ += dS_hf K_hf, 16 keys per step
+            tc::mma_ts(tdQ, tS(hf) + 8u * k, tc::sw128_desc(sK(ks) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024),
+                       idMN, (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+          if (hf == 1) {
+            tc::mma_commit(b_kempty(ks));
+            tc::mma_commit(b_vempty(vs));
+          }
+          if (n + 1 < nsteps) {
+            if (hf == 0 && !wait_kv(n + 1)) { ok = false; break; }
+            tc::tc_fence_after();
+            issue_sd(n + 1, hf);
+          }
+        }
       }
       tc::mma_commit(b_drain);
       volatile int no_abort = 0;
@@ -235,8 +247,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
     int n = 0;
     bool ok = true;
     for (; kt.valid(); kt.next(), ++n) {
-      const int b = n & 1;
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_sd(b), (uint32_t)(n >> 1) & 1u, abort, limit))) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_sd(half), (uint32_t)n & 1u, abort, limit))) {
         ok = false;
         break;
       }
@@ -245,8 +256,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       uint32_t sv[2][32], pv[2][32];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        tc::tmem_ld32(tS(b) + lane_off + 64u * half + 32u * cc, sv[cc]);
-        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, pv[cc]);
+        tc::tmem_ld32(tS(half) + lane_off + 32u * cc, sv[cc]);
+        tc::tmem_ld32(tP(half) + lane_off + 32u * cc, pv[cc]);
       }
       tc::tmem_ld_wait();
 #pragma unroll
@@ -259,11 +270,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
           const float p1 = (c0 + 1 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e + 1]), sl2, -lse2)) : 0.f;
           pk[e] = pack_bf16(p0 * (__uint_as_float(pv[cc][2 * e]) - dl), p1 * (__uint_as_float(pv[cc][2 * e + 1]) - dl));
         }
-        tc::tmem_st16(tS(b) + lane_off + 64u * half + 16u * cc, pk);
+        tc::tmem_st16(tS(half) + lane_off + 16u * cc, pk);
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
-      tc::mbar_arrive(b_ds(b));
+      tc::mbar_arrive(b_ds(half));
     }
     if (__all_sync(0xffffffffu, ok && !*abort) && vrow) {
       bool have = n > 0;
@@ -331,12 +342,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
   const uint32_t b_kv = sBar;
   auto b_qfull = [&](int s) { return sBar + 8u * (1 + s); };    // Q_n and dO_n landed
   auto b_qempty = [&](int s) { return sBar + 8u * (3 + s); };
-  const uint32_t b_st = sBar + 8u * 5;     // S^T_n and dP^T_n done
-  const uint32_t b_p = sBar + 8u * 6;      // P^T_n in TMEM, dS^T_n in smem (128 arrivals)
-  const uint32_t b_dsfree = sBar + 8u * 7; // dK_n finished reading dS^T
-  const uint32_t b_drain = sBar + 8u * 8;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 10);
-  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 10 + 4);
+  auto b_st = [&](int hf) { return sBar + 8u * (5 + hf); };      // S^T, dP^T of query half hf done
+  auto b_p = [&](int hf) { return sBar + 8u * (7 + hf); };       // P^T, dS^T of half hf ready (128 arrivals)
+  auto b_dsfree = [&](int hf) { return sBar + 8u * (9 + hf); };  // dK finished reading dS^T half hf
+  const uint32_t b_drain = sBar + 8u * 11;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 12);
+  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 12 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -352,9 +363,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
       tc::mbar_init(b_qfull(s), 1);
       tc::mbar_init(b_qempty(s), 1);
     }
-    tc::mbar_init(b_st, 1);
-    tc::mbar_init(b_p, 256);
-    tc::mbar_init(b_dsfree, 1);
+    for (int hf = 0; hf < 2; ++hf) {
+      tc::mbar_init(b_st(hf), 1);
+      tc::mbar_init(b_p(hf), 128);
+      tc::mbar_init(b_dsfree(hf), 1);
+    }
     tc::mbar_init(b_drain, 1);
     *abort = 0;
     tc::fence_barrier_init();
@@ -367,7 +380,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tdK = tmem, tdV = tmem + 128, tS = tmem + 256, tdP = tmem + 384;
+  // dK | dV | S^T half A | S^T half B | dP^T half A | dP^T half B  (halves: queries 0-63, 64-127)
+  const uint32_t tdK = tmem, tdV = tmem + 128;
+  auto tS = [&](int hf) { return tmem + 256u + 64u * (uint32_t)hf; };
+  auto tP = [&](int hf) { return tmem + 384u + 64u * (uint32_t)hf; };
   const uint32_t limit = args.wait_limit;
 
   if (warp == 0) {
@@ -404,38 +420,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
   } else if (warp == 1) {
     if (lane == 0) {
       const int nsteps = count_key_tiles(args.row_idx, args.blocks, e0, e1);
-      constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);
+      constexpr uint32_t idH = tc::idesc_bf16(128, 64, false, false);    // S^T, dP^T halves: N = 64 queries
+      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);   // dV, dK: B MN-major
       bool ok = tc::mbar_wait(b_kv, 0, abort, limit);
-      for (int n = 0; ok && n < nsteps; ++n) {
+      // S^T_hf = K Q_hf^T and dP^T_hf = V dO_hf^T for query half hf of tile n
+      auto issue_st = [&](int n, int hf) {
         const int s = n % kKvQStages;
-        if (!tc::mbar_wait(b_qfull(s), (uint32_t)(n / kKvQStages) & 1u, abort, limit)) break;
-        tc::tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {   // S^T = K Q^T ; dP^T = V dO^T
+        for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tS, tc::sw128_desc(sK + off, 16, 1024), tc::sw128_desc(sQ(s) + off, 16, 1024), idNT, k > 0);
+          tc::mma_ss(tS(hf), tc::sw128_desc(sK + off, 16, 1024), tc::sw128_desc(sQ(s) + 8192u * hf + off, 16, 1024),
+                     idH, k > 0);
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tdP, tc::sw128_desc(sV + off, 16, 1024), tc::sw128_desc(sO(s) + off, 16, 1024), idNT, k > 0);
+          tc::mma_ss(tP(hf), tc::sw128_desc(sV + off, 16, 1024), tc::sw128_desc(sO(s) + 8192u * hf + off, 16, 1024),
+                     idH, k > 0);
         }
-        tc::mma_commit(b_st);
-        if (!tc::mbar_wait(b_p, (uint32_t)n & 1u, abort, limit)) break;
-        tc::tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < 8; ++k)   // dV += P^T dO, 16 queries per step
-          tc::mma_ts(tdV, tS + half_col(k), tc::sw128_desc(sO(s) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
-                     (n > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {  // dK += dS^T Q
-          const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tdK, tc::sw128_desc(sdS + off, 16, 1024),
-                     tc::sw128_desc(sQ(s) + 2048u * k, kTcTileBytes / 2, 1024), idMN, (n > 0 || k > 0) ? 1u : 0u);
+        tc::mma_commit(b_st(hf));
+      };
+      if (ok && nsteps > 0) {
+        ok = tc::mbar_wait(b_qfull(0), 0, abort, limit);
+        if (ok) {
+          tc::tc_fence_after();
+          issue_st(0, 0);
+          issue_st(0, 1);
         }
-        tc::mma_commit(b_dsfree);
-        tc::mma_commit(b_qempty(s));
+      }
+      for (int n = 0; ok && n < nsteps; ++n) {
+        const int s = n % kKvQStages;
+        for (int hf = 0; hf < 2 && ok; ++hf) {
+          if (!tc::mbar_wait(b_p(hf), (uint32_t)n & 1u, abort, limit)) { ok = false; break; }
+          tc::tc_fence_after();
+          const uint32_t acc0 = (n > 0 || hf > 0) ? 1u : 0u;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)   // dV += P^T_hf dO_hf, 16 queries per step
+            tc::mma_ts(tdV, tS(hf) + 8u * k, tc::sw128_desc(sO(s) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024),
+                       idMN, (acc0 || k > 0) ? 1u : 0u);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)   // dK += dS^T_hf Q_hf
+            tc::mma_ss(tdK, tc::sw128_desc(sdS + (uint32_t)hf * (kTcTileBytes / 2) + 32u * k, 16, 1024),
+                       tc::sw128_desc(sQ(s) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024), idMN,
+                       (acc0 || k > 0) ? 1u : 0u);
+          tc::mma_commit(b_dsfree(hf));
+          if (hf == 1) tc::mma_commit(b_qempty(s));
+          if (n + 1 < nsteps) {
+            if (hf == 0 && !tc::mbar_wait(b_qfull((n + 1) % kKvQStages), (uint32_t)((n + 1) / kKvQStages) & 1u,
+                                          abort, limit)) {
+              ok = false;
+              break;
+            }
+            tc::tc_fence_after();
+            issue_st(n + 1, hf);
+          }
+        }
       }
       tc::mma_commit(b_drain);
       volatile int no_abort = 0;
@@ -462,11 +501,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
       }
       const float4 *st_l = reinterpret_cast<const float4 *>(sgen + (sStat(s) - sbase)) + 16 * half;
       const float4 *st_d = st_l + 32;
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_st, (uint32_t)n & 1u, abort, limit))) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_st(half), (uint32_t)n & 1u, abort, limit))) {
         ok = false;
         break;
       }
-      if (n > 0 && !__all_sync(0xffffffffu, tc::mbar_wait(b_dsfree, (uint32_t)(n - 1) & 1u, abort, limit))) {
+      if (n > 0 &&
+          !__all_sync(0xffffffffu, tc::mbar_wait(b_dsfree(half), (uint32_t)(n - 1) & 1u, abort, limit))) {
         ok = false;
         break;
       }
@@ -474,8 +514,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
       uint32_t sv[2][32], pv[2][32];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        tc::tmem_ld32(tS + lane_off + 64u * half + 32u * cc, sv[cc]);
-        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, pv[cc]);
+        tc::tmem_ld32(tS(half) + lane_off + 32u * cc, sv[cc]);
+        tc::tmem_ld32(tP(half) + lane_off + 32u * cc, pv[cc]);
       }
       tc::tmem_ld_wait();
       const bool full = qv >= 64 * half + 64;   // no padding columns in this half
@@ -503,7 +543,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
           dk[2 * g + 1] = pack_bf16(p2 * (__uint_as_float(pv[cc][4 * g + 2]) - Dv.z),
                                     p3 * (__uint_as_float(pv[cc][4 * g + 3]) - Dv.w));
         }
-        tc::tmem_st16(tS + lane_off + 64u * half + 16u * cc, pk);
+        tc::tmem_st16(tS(half) + lane_off + 16u * cc, pk);
         // dS^T row into the 128-byte-swizzled K-major tile: this half's 64
         // columns are the half-tile `half`; columns 32cc..32cc+31 of it are
         // 16-byte chunks 4cc..4cc+3
@@ -517,7 +557,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
       tc::tmem_st_wait();
       fence_proxy_async_smem();
       tc::tc_fence_before();
-      tc::mbar_arrive(b_p);
+      tc::mbar_arrive(b_p(half));
     }
     if (__all_sync(0xffffffffu, ok && !*abort) && row < zt.rows) {
       bool have = n > 0;
