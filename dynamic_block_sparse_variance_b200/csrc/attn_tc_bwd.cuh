@@ -93,8 +93,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   auto b_kempty = [&](int s) { return sBar + 8u * (4 + s); };   // 3
   auto b_vfull = [&](int s) { return sBar + 8u * (7 + s); };    // 2
   auto b_vempty = [&](int s) { return sBar + 8u * (9 + s); };   // 2
-  auto b_sd = [&](int hf) { return sBar + 8u * (11 + hf); };     // S and dP of key half hf done
-  auto b_ds = [&](int hf) { return sBar + 8u * (13 + hf); };     // dS of key half hf written (128 arrivals)
+  auto b_sd = [&](int b) { return sBar + 8u * (11 + b); };      // S_n and dP_n done
+  auto b_ds = [&](int b) { return sBar + 8u * (13 + b); };      // dS_n written (128 arrivals)
   const uint32_t b_drain = sBar + 8u * 15;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 16);
   volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 16 + 4);
@@ -117,9 +117,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       tc::mbar_init(b_vfull(s), 1);
       tc::mbar_init(b_vempty(s), 1);
     }
-    for (int hf = 0; hf < 2; ++hf) {
-      tc::mbar_init(b_sd(hf), 1);
-      tc::mbar_init(b_ds(hf), 128);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(b_sd(b), 1);
+      tc::mbar_init(b_ds(b), 256);
     }
     tc::mbar_init(b_drain, 1);
     *abort = 0;
@@ -133,10 +133,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // dQ | S half A | S half B | dP half A | dP half B  (halves: keys 0-63, 64-127)
-  const uint32_t tdQ = tmem;
-  auto tS = [&](int hf) { return tmem + 128u + 64u * (uint32_t)hf; };
-  auto tP = [&](int hf) { return tmem + 256u + 64u * (uint32_t)hf; };
+  auto tS = [&](int b) { return tmem + 128u * (uint32_t)b; };
+  const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
   const uint32_t limit = args.wait_limit;
 
   if (warp == 0) {
@@ -176,57 +174,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   } else if (warp == 1) {
     if (lane == 0) {
       const int nsteps = count_key_tiles(args.col, args.blocks, e0, e1);
-      constexpr uint32_t idH = tc::idesc_bf16(128, 64, false, false);    // S, dP halves: N = 64 keys
-      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);   // dQ: B MN-major
+      constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
+      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);    // B MN-major
       bool ok = tc::mbar_wait(b_q, 0, abort, limit);
-      // S_hf = Q K_hf^T and dP_hf = dO V_hf^T for key half hf of tile n
-      auto issue_sd = [&](int n, int hf) {
-        const int ks = n % kDqKStages, vs = n % kDqVStages;
+      auto issue_s = [&](int n) -> bool {   // S_n = Q K_n^T
+        const int ks = n % kDqKStages;
+        if (!tc::mbar_wait(b_kfull(ks), (uint32_t)(n / kDqKStages) & 1u, abort, limit)) return false;
+        tc::tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tS(hf), tc::sw128_desc(sQ + off, 16, 1024),
-                     tc::sw128_desc(sK(ks) + 8192u * hf + off, 16, 1024), idH, k > 0);
+          tc::mma_ss(tS(n & 1), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK(ks) + off, 16, 1024), idNT,
+                     k > 0);
         }
+        return true;
+      };
+      auto issue_dp = [&](int n) -> bool {   // dP_n = dO V_n^T
+        const int vs = n % kDqVStages;
+        if (!tc::mbar_wait(b_vfull(vs), (uint32_t)(n / kDqVStages) & 1u, abort, limit)) return false;
+        tc::tc_fence_after();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tP(hf), tc::sw128_desc(sO + off, 16, 1024),
-                     tc::sw128_desc(sV(vs) + 8192u * hf + off, 16, 1024), idH, k > 0);
+          tc::mma_ss(tdP, tc::sw128_desc(sO + off, 16, 1024), tc::sw128_desc(sV(vs) + off, 16, 1024), idNT,
+                     k > 0);
         }
-        tc::mma_commit(b_sd(hf));
+        tc::mma_commit(b_vempty(vs));
+        tc::mma_commit(b_sd(n & 1));
+        return true;
       };
-      auto wait_kv = [&](int n) -> bool {
-        return tc::mbar_wait(b_kfull(n % kDqKStages), (uint32_t)(n / kDqKStages) & 1u, abort, limit) &&
-               tc::mbar_wait(b_vfull(n % kDqVStages), (uint32_t)(n / kDqVStages) & 1u, abort, limit);
-      };
-      if (ok && nsteps > 0) {
-        ok = wait_kv(0);
-        if (ok) {
-          tc::tc_fence_after();
-          issue_sd(0, 0);
-          issue_sd(0, 1);
-        }
-      }
+      if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
       for (int n = 0; ok && n < nsteps; ++n) {
-        const int ks = n % kDqKStages, vs = n % kDqVStages;
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          if (!tc::mbar_wait(b_ds(hf), (uint32_t)n & 1u, abort, limit)) { ok = false; break; }
-          tc::tc_fence_after();
+        if (n + 1 < nsteps && !issue_s(n + 1)) break;
+        if (!tc::mbar_wait(b_ds(n & 1), (uint32_t)(n >> 1) & 1u, abort, limit)) break;
+        tc::tc_fence_after();
+        if (n + 1 < nsteps && !issue_dp(n + 1)) break;
+        const int ks = n % kDqKStages;
 #pragma unroll
-          for (int k = 0; k < 4; ++k)   // dQ += dS_hf K_hf, 16 keys per step
-            tc::mma_ts(tdQ, tS(hf) + 8u * k, tc::sw128_desc(sK(ks) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024),
-                       idMN, (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
-          if (hf == 1) {
-            tc::mma_commit(b_kempty(ks));
-            tc::mma_commit(b_vempty(vs));
-          }
-          if (n + 1 < nsteps) {
-            if (hf == 0 && !wait_kv(n + 1)) { ok = false; break; }
-            tc::tc_fence_after();
-            issue_sd(n + 1, hf);
-          }
-        }
+        for (int k = 0; k < 8; ++k)   // dQ += dS_n K_n, 16 keys per step
+          tc::mma_ts(tdQ, tS(n & 1) + half_col(k), tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
+                     (n > 0 || k > 0) ? 1u : 0u);
+        tc::mma_commit(b_kempty(ks));
       }
       tc::mma_commit(b_drain);
       volatile int no_abort = 0;
@@ -247,7 +235,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
     int n = 0;
     bool ok = true;
     for (; kt.valid(); kt.next(), ++n) {
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_sd(half), (uint32_t)n & 1u, abort, limit))) {
+      const int b = n & 1;
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_sd(b), (uint32_t)(n >> 1) & 1u, abort, limit))) {
         ok = false;
         break;
       }
@@ -256,8 +245,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       uint32_t sv[2][32], pv[2][32];
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        tc::tmem_ld32(tS(half) + lane_off + 32u * cc, sv[cc]);
-        tc::tmem_ld32(tP(half) + lane_off + 32u * cc, pv[cc]);
+        tc::tmem_ld32(tS(b) + lane_off + 64u * half + 32u * cc, sv[cc]);
+        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, pv[cc]);
       }
       tc::tmem_ld_wait();
 #pragma unroll
@@ -270,11 +259,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
           const float p1 = (c0 + 1 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e + 1]), sl2, -lse2)) : 0.f;
           pk[e] = pack_bf16(p0 * (__uint_as_float(pv[cc][2 * e]) - dl), p1 * (__uint_as_float(pv[cc][2 * e + 1]) - dl));
         }
-        tc::tmem_st16(tS(half) + lane_off + 16u * cc, pk);
+        tc::tmem_st16(tS(b) + lane_off + 64u * half + 16u * cc, pk);
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
-      tc::mbar_arrive(b_ds(half));
+      tc::mbar_arrive(b_ds(b));
     }
     if (__all_sync(0xffffffffu, ok && !*abort) && vrow) {
       bool have = n > 0;
