@@ -5,6 +5,7 @@
 
 #include <cmath>
 #include <cstdio>
+#include <mutex>
 #include <string>
 
 #include "attn_mma_bwd.cuh"
@@ -241,6 +242,76 @@ int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, cons
                                                     d.ZX, part));
   PRISM_TRACED("zone_finish_kernel", st, zone_finish_kernel<<<(unsigned)d.Z, 64, 0, st>>>(part, w.nslab, (int)d.C, audio, d.H, d.W, d.ZY, d.ZX, rec));
   PRISM_TRACED("zone_final_kernel", st, zone_final_kernel<<<1, 1024, 0, st>>>(rec, (int)d.Z, audio != nullptr, p->eps, g, rho, debug));
+  PRISM_CUDA_CHECK_LAUNCH();
+  return PRISM_OK;
+}
+
+}  // extern "C"
+
+// Scratch of prism_zone_indicator_noalloc: partial sums for up to
+// PRISM_NOALLOC_MAX_ZONES zones x PRISM_NOALLOC_MAX_CHANNELS channels, laid
+// out exactly like the indicator workspace.  Host code must not pass this
+// name to a kernel (on the host it is only a stand-in); the device address is
+// looked up once per device below.
+constexpr size_t kNoallocPartBytes =
+    (size_t)PRISM_NOALLOC_MAX_ZONES * (PRISM_NOALLOC_MAX_CHANNELS / kSlab) * 3 * sizeof(float);
+constexpr size_t kNoallocBytes = kNoallocPartBytes + (size_t)PRISM_NOALLOC_MAX_ZONES * kZoneRec * sizeof(double);
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocBytes];
+
+static std::mutex g_noalloc_mutex;
+static void *g_noalloc_addr[256];   // per device ordinal
+
+// Device address of the fixed scratch on the current device (looked up on the
+// first call for that device).
+static int noalloc_scratch(void **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(PRISM_ECUDA, cudaGetErrorString(e));
+  if (dev < 0 || dev >= 256) return fail(PRISM_EINVAL, "device ordinal out of range");
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void *ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return fail(PRISM_ECUDA, cudaGetErrorString(e));
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return PRISM_OK;
+}
+
+extern "C" {
+
+int prism_zone_indicator_noalloc(const prism_params *p, const void *V, int v_dtype, const float *audio, float *g,
+                                 float *rho, float *debug, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!V || !g || !rho) return fail(PRISM_EINVAL, "V, g and rho must be non-NULL");
+  if (!aligned16(V)) return fail(PRISM_EINVAL, "V must be 16-byte aligned");
+  if (v_dtype != PRISM_BF16 && v_dtype != PRISM_F32) return fail(PRISM_EINVAL, "V dtype must be bf16 or f32");
+  if (d.Z > PRISM_NOALLOC_MAX_ZONES || d.C > PRISM_NOALLOC_MAX_CHANNELS)
+    return fail(PRISM_EINVAL, "grid too large for the fixed scratch (see PRISM_NOALLOC_MAX_*)");
+  IndicatorWs w(d);
+  if (w.total > kNoallocBytes) return fail(PRISM_EINVAL, "grid too large for the fixed scratch");
+  void *scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  cudaStream_t st = as_stream(stream);
+  uint8_t *ws = static_cast<uint8_t *>(scratch);
+  // every partial and record is written before it is read, so nothing needs clearing
+  float *part = reinterpret_cast<float *>(ws + w.part);
+  double *rec = reinterpret_cast<double *>(ws + w.rec);
+  dim3 grid(w.nslab, (unsigned)d.Z);
+  if (v_dtype == PRISM_BF16)
+    PRISM_TRACED("zone_stats_kernel", st, zone_stats_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16 *>(V), (int)d.C, d.H, d.W, d.ZY, d.ZX, part));
+  else
+    PRISM_TRACED("zone_stats_kernel", st, zone_stats_kernel<float><<<grid, 256, 0, st>>>(
+        static_cast<const float *>(V), (int)d.C, d.H, d.W, d.ZY, d.ZX, part));
+  PRISM_TRACED("zone_finish_kernel", st, zone_finish_kernel<<<(unsigned)d.Z, 64, 0, st>>>(
+      part, w.nslab, (int)d.C, audio, d.H, d.W, d.ZY, d.ZX, rec));
+  PRISM_TRACED("zone_final_kernel", st, zone_final_kernel<<<1, 1024, 0, st>>>(rec, (int)d.Z, audio != nullptr,
+                                                                                p->eps, g, rho, debug));
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
 }

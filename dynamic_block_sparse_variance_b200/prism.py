@@ -23,7 +23,8 @@ PRISM_OPT_ATTN_BACKEND, PRISM_OPT_WAIT_LIMIT, PRISM_OPT_DEBUG_STALL = 0, 1, 2
 
 # Entry points declared in include/prism.h, in declaration order.
 ENTRY_POINTS = (
-    "prism_workspace_size", "prism_zone_indicator", "prism_assign_blocks", "prism_permute",
+    "prism_workspace_size", "prism_zone_indicator", "prism_zone_indicator_noalloc", "prism_assign_blocks",
+    "prism_permute",
     "prism_unpermute", "prism_block_select", "prism_bsa_fwd", "prism_bsa_bwd",
     "prism_set_option", "prism_set_trace", "prism_device_status", "prism_last_error",
 )
@@ -69,6 +70,7 @@ def lib():
         sig = {
             "prism_workspace_size": [pp, ctypes.c_int, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)],
             "prism_zone_indicator": [pp, _P, ctypes.c_int, _P, _P, _P, _P, _P, sz, _P],
+            "prism_zone_indicator_noalloc": [pp, _P, ctypes.c_int, _P, _P, _P, _P, _P],
             "prism_assign_blocks": [pp, _P, _P, _P, _P, _P, _P, _P],
             "prism_permute": [pp, _P, _P, _P, ctypes.c_int, _P, _P, _P],
             "prism_unpermute": [pp, _P, _P, ctypes.c_int, _P, ctypes.c_int, _P],
@@ -121,6 +123,12 @@ def prism_workspace_size(p, kind, col_capacity=0):
 def prism_zone_indicator(p, V, audio, g, rho, debug, workspace):
     _check(lib().prism_zone_indicator(ctypes.byref(p), _ptr(V), _dtype(V), _ptr(audio), _ptr(g), _ptr(rho),
                                       _ptr(debug), _ptr(workspace), workspace.numel(), _stream()))
+
+
+def prism_zone_indicator_noalloc(p, V, audio, g, rho, debug=None):
+    """The indicator with no workspace argument (fixed scratch inside the library)."""
+    _check(lib().prism_zone_indicator_noalloc(ctypes.byref(p), _ptr(V), _dtype(V), _ptr(audio), _ptr(g), _ptr(rho),
+                                              _ptr(debug), _stream()))
 
 
 def prism_assign_blocks(p, g, rho, shape_id, zone_blk_base, blocks, nblk):

@@ -118,6 +118,31 @@ int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, cons
                          prism_stream stream);
 
 /*
+ * prism_zone_indicator without any workspace: the same computation, with its
+ * scratch (per-zone partial sums) held in a fixed device array inside the
+ * library.  It is for callers that cannot allocate device memory at the
+ * point of the call: plugins that run inside another framework's execution
+ * (which hands them only the input and output buffers), allocator-free or
+ * real-time runtimes that must not block on cudaMalloc's implicit device
+ * synchronisation, and code that otherwise would have to keep a workspace
+ * alive between calls.  The pages have no counterpart; it is a deployment aid.
+ *   Limits: at most PRISM_NOALLOC_MAX_ZONES macro-zones and at most
+ *   PRISM_NOALLOC_MAX_CHANNELS channels (heads * head_dim); larger problems
+ *   return PRISM_EINVAL without launching anything.
+ *   The fixed array (about 1.8 MiB) is reserved on every GPU that loads the
+ *   library until the process exits.  The first call on each device looks up
+ *   the array's device address (cudaGetSymbolAddress) with that device
+ *   current; make that first call before any stream capture.  All calls share
+ *   the one array: calls that overlap on the GPU (different streams, or
+ *   different host threads, without ordering between them) race on it.
+ *   Every other argument, layout and error behaves as in prism_zone_indicator.
+ */
+#define PRISM_NOALLOC_MAX_ZONES 4096
+#define PRISM_NOALLOC_MAX_CHANNELS 4096
+int prism_zone_indicator_noalloc(const prism_params *p, const void *V, int v_dtype, const float *audio,
+                                 float *g, float *rho, float *debug, prism_stream stream);
+
+/*
  * Method §2: block volume B(m) (rho >= tau128 -> 64, tau256 <= rho < tau128 ->
  * 128, else 256), optimal log2 edges l*_d = -1/2 log2 g_d + 1/3(S + 1/2 sum
  * log2 g), and the nearest of the 16 candidate shapes (edges in {2,4,8},
