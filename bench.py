@@ -104,27 +104,30 @@ class ClockSampler:
 
 # ------------------------------------------------------------- counting --
 def executed_pairs(att):
-    """sum over heads, query blocks i and selected key blocks j of B_i * B_j."""
+    """sum over heads, query blocks i and selected key blocks j of B_i * B_j
+    (in total, and for query blocks of 256 tokens alone)."""
     nb = int(att.nblk.item())
     sizes = att.blocks[:nb, 1].to(torch.int64)
     nnz = int(att.nnz.item())
-    total = 0
+    total = big = 0
     for h in range(att.heads):
         rp = att.row_ptr[h * att.cap: h * att.cap + nb + 1].to(torch.int64)
         cnt = rp[1:] - rp[:-1]
         cols = att.col[int(rp[0]): int(rp[-1])].to(torch.int64)
         rows = torch.repeat_interleave(torch.arange(nb, device=cols.device), cnt)
-        total += int((sizes[rows] * sizes[cols]).sum().item())
-    return total, nnz, nb, sizes
+        prod = sizes[rows] * sizes[cols]
+        total += int(prod.sum().item())
+        big += int(prod[sizes[rows] == 256].sum().item())
+    return total, nnz, nb, sizes, big
 
 
 # Algorithmic tensor-core FLOPs of each attention kernel, in units of
 # P = sum_h sum_i sum_{j in S_i} B_i B_j d: forward 4P (QK^T, PV); the key-side
 # backward kernel 8P (S, dP, dV, dK); the query-side one 2P (dQ; its S and dP
 # recomputation is extra work and not counted).
-KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_fwd_tc_kernel": 4, "bsa_dkdv_mma_kernel": 8,
+KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_fwd_tc_kernel": 4, "bsa_fwd_tc2_kernel": 4, "bsa_dkdv_mma_kernel": 8,
                      "bsa_dkdv_tc_kernel": 8, "bsa_dq_mma_kernel": 2, "bsa_dq_tc_kernel": 2}
-FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel")
+FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
 BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel", "bsa_dkdv_tc_kernel", "bsa_dq_tc_kernel")
 
 
@@ -250,8 +253,11 @@ def run_prism(args, rank, world):
     for _ in range(args.warmup):
         step()
     P.prism_device_status()
-    pairs, nnz, nb, sizes = executed_pairs(att)
+    pairs, nnz, nb, sizes, pairs256 = executed_pairs(att)
     Punit = float(pairs) * wl.head_dim
+    # work of each forward kernel: the paired kernel takes the 256-token query blocks
+    unit_of = {"bsa_fwd_tc2_kernel": float(pairs256) * wl.head_dim,
+               "bsa_fwd_tc_kernel": float(pairs - pairs256) * wl.head_dim}
     exec_flops = 14.0 * Punit
     dense_flops = 14.0 * float(wl.N) ** 2 * wl.head_dim * wl.heads
 
@@ -280,7 +286,8 @@ def run_prism(args, rank, world):
     dom = max(summ.items(), key=lambda kv: kv[1][1])
     dom_name, (dom_n, dom_ms) = dom
     if dom_name in KERNEL_FLOP_UNITS:
-        per_launch = KERNEL_FLOP_UNITS[dom_name] * Punit
+        split = "bsa_fwd_tc2_kernel" in summ
+        per_launch = KERNEL_FLOP_UNITS[dom_name] * (unit_of[dom_name] if split and dom_name in unit_of else Punit)
         achieved = per_launch / (dom_ms / dom_n * 1e-3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
         roof = dict(kernel=dom_name, bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",

@@ -35,6 +35,7 @@ struct TcFwdArgs {
   float *lse;
   uint32_t wait_limit;
   int debug_stall;   // test knob: the softmax never signals P_0, so the MMA wait times out
+  int skip256;       // zones of 256-token blocks are left to the paired kernel
 };
 
 // Iterates the 128-key sub-tiles of the key blocks col[e0..e1).
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
   const int b0 = args.zone_blk_base[m];
   const int B = args.blocks[b0].size;
   if (B >= 128 && t >= 4) return;  // zones of 128/256 blocks hold four 128-row tiles
+  if (B == 256 && args.skip256) return;
   int qb, r0, qrows;
   if (B == 64) {
     qb = b0 + t;
@@ -330,6 +332,304 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
           uint32_t ov[32];
           if (nsteps > 0) {
             tc::tmem_ld32(tO + lane_off + 32u * c, ov);
+            tc::tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = 0u;
+          }
+#pragma unroll
+          for (int v8 = 0; v8 < 4; ++v8) {
+            uint4 u, r;
+            uint32_t *up = &u.x, *rp = &r.x;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x0 = __uint_as_float(ov[8 * v8 + 2 * e]) * inv;
+              const float x1 = __uint_as_float(ov[8 * v8 + 2 * e + 1]) * inv;
+              up[e] = pack_bf16(x0, x1);
+              rp[e] = pack_bf16(x0 - bf16_lo(up[e]), x1 - bf16_hi(up[e]));
+            }
+            *reinterpret_cast<uint4 *>(orow + 32 * c + 8 * v8) = u;
+            if (rrow) *reinterpret_cast<uint4 *>(rrow + 32 * c + 8 * v8) = r;
+          }
+        }
+        args.lse[orow_idx] = (nsteps > 0 && l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+      }
+    }
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace prism
+
+namespace prism {
+
+// ---------------------------------------------------------------------------
+// Paired forward: one CTA per (256-token query block, head).  The block's two
+// 128-row tiles A and B share every K/V tile (one TMA load serves both), and
+// their softmax warp groups ping-pong with the MMA issuer:
+//   S_A(0) S_B(0) | PV_A(0) S_A(1) PV_B(0) S_B(1) | PV_A(1) S_A(2) ...
+// so one tile's softmax runs while the other tile's MMAs execute.
+// TMEM: S_A | O_A | S_B | O_B.  S_g(n+1) is issued after PV_g(n), hence its
+// completion also proves PV_g(n) complete, which is what the lazy O rescale
+// of step n+1 needs.
+constexpr int kTc2Stages = 2;
+constexpr int kTc2SmemBytes = kTcTileBytes * (2 + 2 * kTc2Stages) + 256 + 1024;
+constexpr int kTc2Threads = 320;   // producer, MMA, 2 x 4 softmax warps
+
+__global__ void __maxnreg__(200) bsa_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                                     const __grid_constant__ CUtensorMap tmK,
+                                                                     const __grid_constant__ CUtensorMap tmV,
+                                                                     const TcFwdArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  uint8_t *sgen = smem_raw + (sbase - smem_u32(smem_raw));
+  auto sQ = [&](int g) { return sbase + (uint32_t)g * kTcTileBytes; };
+  auto sK = [&](int s) { return sbase + (uint32_t)(2 + 2 * s) * kTcTileBytes; };
+  auto sV = [&](int s) { return sbase + (uint32_t)(3 + 2 * s) * kTcTileBytes; };
+  const uint32_t sBar = sbase + (uint32_t)(2 + 2 * kTc2Stages) * kTcTileBytes;
+  const uint32_t b_q = sBar;
+  auto b_kfull = [&](int s) { return sBar + 8u * (1 + s); };
+  auto b_vfull = [&](int s) { return sBar + 8u * (3 + s); };
+  auto b_kempty = [&](int s) { return sBar + 8u * (5 + s); };
+  auto b_vempty = [&](int s) { return sBar + 8u * (7 + s); };
+  auto b_sfull = [&](int g) { return sBar + 8u * (9 + g); };
+  auto b_pfull = [&](int g) { return sBar + 8u * (11 + g); };
+  const uint32_t b_drain = sBar + 8u * 13;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 14);
+  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 14 + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int m = blockIdx.x >> 1, t = blockIdx.x & 1;
+  const int b0 = args.zone_blk_base[m];
+  if (args.blocks[b0].size != 256) return;   // zones of 64/128 blocks run in the single-tile kernel
+  const int qb = b0 + t;
+  const int r0 = m * kZoneTokens + 256 * t;
+  const int e0 = args.row_ptr[(int64_t)h * args.cap + qb];
+  const int e1 = args.row_ptr[(int64_t)h * args.cap + qb + 1];
+  const int row_base = (int)((int64_t)h * args.N);
+
+  if (threadIdx.x == 0) {
+    tc::mbar_init(b_q, 1);
+    for (int s = 0; s < kTc2Stages; ++s) {
+      tc::mbar_init(b_kfull(s), 1);
+      tc::mbar_init(b_vfull(s), 1);
+      tc::mbar_init(b_kempty(s), 1);
+      tc::mbar_init(b_vempty(s), 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      tc::mbar_init(b_sfull(g), 1);
+      tc::mbar_init(b_pfull(g), 128);
+    }
+    tc::mbar_init(b_drain, 1);
+    *abort = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(smem_u32(tmem_slot), 512);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto tS = [&](int g) { return tmem + 256u * (uint32_t)g; };
+  auto tO = [&](int g) { return tmem + 256u * (uint32_t)g + 128u; };
+  const uint32_t limit = args.wait_limit;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmQ);
+      tc::prefetch_tmap(&tmK);
+      tc::prefetch_tmap(&tmV);
+      tc::mbar_expect_tx(b_q, 2 * kTcTileBytes);
+      for (int g = 0; g < 2; ++g) {
+        tc::tma_load_2d(sQ(g), &tmQ, 0, row_base + r0 + 128 * g, b_q);
+        tc::tma_load_2d(sQ(g) + kTcTileBytes / 2, &tmQ, 64, row_base + r0 + 128 * g, b_q);
+      }
+      KeyTiles kt;
+      kt.init(args.col, args.blocks, e0, e1);
+      int nk = 0, nv = 0;
+      for (; kt.valid(); kt.next()) {
+        const int s = nk % kTc2Stages;
+        const uint32_t ph = (uint32_t)(nk / kTc2Stages) & 1u;
+        if (!tc::mbar_wait(b_kempty(s), ph ^ 1u, abort, limit)) break;
+        tc::mbar_expect_tx(b_kfull(s), kTcTileBytes);
+        tc::tma_load_2d(sK(s), &tmK, 0, row_base + kt.row(), b_kfull(s));
+        tc::tma_load_2d(sK(s) + kTcTileBytes / 2, &tmK, 64, row_base + kt.row(), b_kfull(s));
+        ++nk;
+        if (!tc::mbar_wait(b_vempty(s), ph ^ 1u, abort, limit)) break;
+        tc::mbar_expect_tx(b_vfull(s), kTcTileBytes);
+        tc::tma_load_2d(sV(s), &tmV, 0, row_base + kt.row(), b_vfull(s));
+        tc::tma_load_2d(sV(s) + kTcTileBytes / 2, &tmV, 64, row_base + kt.row(), b_vfull(s));
+        ++nv;
+      }
+      volatile int no_abort = 0;
+      tc::mbar_wait(b_q, 0, &no_abort, limit);
+      for (int k = max(0, nk - kTc2Stages); k < nk; ++k)
+        tc::mbar_wait(b_kfull(k % kTc2Stages), (uint32_t)(k / kTc2Stages) & 1u, &no_abort, limit);
+      for (int k = max(0, nv - kTc2Stages); k < nv; ++k)
+        tc::mbar_wait(b_vfull(k % kTc2Stages), (uint32_t)(k / kTc2Stages) & 1u, &no_abort, limit);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const int nsteps = count_key_tiles(args.col, args.blocks, e0, e1);
+      constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idO = tc::idesc_bf16(128, 128, false, true);
+      bool ok = tc::mbar_wait(b_q, 0, abort, limit);
+      auto issue_s = [&](int n, int g) {
+        const int s = n % kTc2Stages;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
+          tc::mma_ss(tS(g), tc::sw128_desc(sQ(g) + off, 16, 1024), tc::sw128_desc(sK(s) + off, 16, 1024), idS,
+                     k > 0);
+        }
+        tc::mma_commit(b_sfull(g));
+      };
+      auto issue_pv = [&](int n, int g) {
+        const int s = n % kTc2Stages;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          tc::mma_ts(tO(g), tS(g) + 8u * k, tc::sw128_desc(sV(s) + 2048u * k, kTcTileBytes / 2, 1024), idO,
+                     (n > 0 || k > 0) ? 1u : 0u);
+      };
+      auto wait_k = [&](int n) {
+        return tc::mbar_wait(b_kfull(n % kTc2Stages), (uint32_t)(n / kTc2Stages) & 1u, abort, limit);
+      };
+      if (ok && nsteps > 0) {
+        ok = wait_k(0);
+        if (ok) {
+          tc::tc_fence_after();
+          issue_s(0, 0);
+          issue_s(0, 1);
+          tc::mma_commit(b_kempty(0));
+        }
+      }
+      for (int n = 0; ok && n < nsteps; ++n) {
+        const int s = n % kTc2Stages;
+        for (int g = 0; g < 2 && ok; ++g) {
+          if (!tc::mbar_wait(b_pfull(g), (uint32_t)n & 1u, abort, limit)) { ok = false; break; }
+          if (g == 0 && !tc::mbar_wait(b_vfull(s), (uint32_t)(n / kTc2Stages) & 1u, abort, limit)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          issue_pv(n, g);
+          if (g == 1) tc::mma_commit(b_vempty(s));
+          if (n + 1 < nsteps) {
+            if (g == 0 && !wait_k(n + 1)) { ok = false; break; }
+            tc::tc_fence_after();
+            issue_s(n + 1, g);
+            if (g == 1) tc::mma_commit(b_kempty((n + 1) % kTc2Stages));
+          }
+        }
+      }
+      tc::mma_commit(b_drain);
+      volatile int no_abort = 0;
+      tc::mbar_wait(b_drain, 0, &no_abort, limit);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int g = (warp - 2) >> 2;           // tile A (rows 0..127) or B (128..255)
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const float sl2 = args.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    KeyTiles kt;
+    kt.init(args.col, args.blocks, e0, e1);
+    int n = 0;
+    bool ok = true;
+    for (; kt.valid(); kt.next(), ++n) {
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_sfull(g), (uint32_t)n & 1u, abort, limit))) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+      uint32_t raw[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_ld32(tS(g) + lane_off + 32u * c, raw[c]);
+      tc::tmem_ld_wait();
+      const int kv = kt.keys();
+      if (kv < 128) {
+#pragma unroll
+        for (int c = 2; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) raw[c][e] = __float_as_uint(-INFINITY);
+      }
+      float m8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      mx *= sl2;
+      const bool grow = mx > m_run + 8.f;
+      const float alpha = grow ? tc::ex2(m_run - mx) : 1.f;
+      if (grow) {
+        l_run *= alpha;
+        m_run = mx;
+      }
+      if (n > 0 && __any_sync(0xffffffffu, grow)) {
+        // S_g(n) was issued after PV_g(n-1): its completion proves O settled
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[32];
+          tc::tmem_ld32(tO(g) + lane_off + 32u * c, ov);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tc::tmem_st32(tO(g) + lane_off + 32u * c, ov);
+        }
+      }
+      float r8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r8[e] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
+          r8[e & 7] += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        tc::tmem_st16(tS(g) + lane_off + 16u * c, pk);
+      }
+      l_run += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(b_pfull(g));
+    }
+    const int nsteps = n;
+    const int64_t orow_idx = (int64_t)h * args.N + r0 + 128 * g + row;
+    if (__all_sync(0xffffffffu, ok && !*abort)) {
+      float inv = 0.f;
+      if (nsteps > 0) {
+        if (__all_sync(0xffffffffu, tc::mbar_wait(b_drain, 0, abort, limit))) {
+          tc::tc_fence_after();
+          inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        } else {
+          ok = false;
+        }
+      }
+      if (ok) {
+        __nv_bfloat16 *orow = args.o + orow_idx * 128;
+        __nv_bfloat16 *rrow = args.o_res ? args.o_res + orow_idx * 128 : nullptr;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ov[32];
+          if (nsteps > 0) {
+            tc::tmem_ld32(tO(g) + lane_off + 32u * c, ov);
             tc::tmem_ld_wait();
           } else {
 #pragma unroll

@@ -479,6 +479,12 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
     a.lse = lse;
     a.wait_limit = g_wait_limit ? g_wait_limit : kDefaultWaitLimit;
     a.debug_stall = g_debug_stall;
+    a.skip256 = g_debug_stall ? 0 : 1;   // the timeout test drives the single-tile kernel alone
+    if (a.skip256) {
+      cudaFuncSetAttribute(bsa_fwd_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTc2SmemBytes);
+      dim3 pgrid((unsigned)(d.Z * 2), d.heads);
+      PRISM_TRACED("bsa_fwd_tc2_kernel", st, bsa_fwd_tc2_kernel<<<pgrid, kTc2Threads, kTc2SmemBytes, st>>>(tq, tk, tv, a));
+    }
     cudaFuncSetAttribute(bsa_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcSmemBytes);
     dim3 tgrid((unsigned)(d.Z * 8), d.heads);
     PRISM_TRACED("bsa_fwd_tc_kernel", st, bsa_fwd_tc_kernel<<<tgrid, 192, kTcSmemBytes, st>>>(tq, tk, tv, a));
