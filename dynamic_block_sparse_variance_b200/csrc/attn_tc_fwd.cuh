@@ -381,7 +381,7 @@ constexpr int kTc2Stages = 2;
 constexpr int kTc2SmemBytes = kTcTileBytes * (2 + 2 * kTc2Stages) + 256 + 1024;
 constexpr int kTc2Threads = 320;   // producer, MMA, 2 x 4 softmax warps
 
-__global__ void __maxnreg__(200) bsa_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ,
+__global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                                      const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV,
                                                                      const TcFwdArgs args) {
@@ -400,8 +400,9 @@ __global__ void __maxnreg__(200) bsa_fwd_tc2_kernel(const __grid_constant__ CUte
   auto b_sfull = [&](int g) { return sBar + 8u * (9 + g); };
   auto b_pfull = [&](int g) { return sBar + 8u * (11 + g); };
   const uint32_t b_drain = sBar + 8u * 13;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 14);
-  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 14 + 4);
+  auto b_pvd = [&](int g) { return sBar + 8u * (14 + g); };    // PV_g(n) complete
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 16);
+  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 16 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -425,6 +426,7 @@ __global__ void __maxnreg__(200) bsa_fwd_tc2_kernel(const __grid_constant__ CUte
     for (int g = 0; g < 2; ++g) {
       tc::mbar_init(b_sfull(g), 1);
       tc::mbar_init(b_pfull(g), 128);
+      tc::mbar_init(b_pvd(g), 1);
     }
     tc::mbar_init(b_drain, 1);
     *abort = 0;
@@ -521,9 +523,12 @@ __global__ void __maxnreg__(200) bsa_fwd_tc2_kernel(const __grid_constant__ CUte
           }
           tc::tc_fence_after();
           issue_pv(n, g);
+          tc::mma_commit(b_pvd(g));
           if (g == 1) tc::mma_commit(b_vempty(s));
           if (n + 1 < nsteps) {
             if (g == 0 && !wait_k(n + 1)) { ok = false; break; }
+            // S_g(n+1) overwrites the columns PV_g(n) reads P from: let PV_g(n) finish first
+            if (!tc::mbar_wait(b_pvd(g), (uint32_t)n & 1u, abort, limit)) { ok = false; break; }
             tc::tc_fence_after();
             issue_s(n + 1, g);
             if (g == 1) tc::mma_commit(b_kempty((n + 1) % kTc2Stages));
@@ -552,24 +557,23 @@ __global__ void __maxnreg__(200) bsa_fwd_tc2_kernel(const __grid_constant__ CUte
         break;
       }
       tc::tc_fence_after();
-      uint32_t raw[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tc::tmem_ld32(tS(g) + lane_off + 32u * c, raw[c]);
-      tc::tmem_ld_wait();
       const int kv = kt.keys();
-      if (kv < 128) {
-#pragma unroll
-        for (int c = 2; c < 4; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) raw[c][e] = __float_as_uint(-INFINITY);
-      }
+      // pass 1: row max over the valid columns, half a row of registers at a time
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int hh = 0; hh < 2; ++hh) {
+        if (hh == 1 && kv <= 64) break;   // a 64-key block: the upper half is padding
+        uint32_t raw[2][32];
+        tc::tmem_ld32(tS(g) + lane_off + 64u * hh, raw[0]);
+        tc::tmem_ld32(tS(g) + lane_off + 64u * hh + 32u, raw[1]);
+        tc::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
+      }
       float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= sl2;
       const bool grow = mx > m_run + 8.f;
@@ -590,16 +594,20 @@ __global__ void __maxnreg__(200) bsa_fwd_tc2_kernel(const __grid_constant__ CUte
           tc::tmem_st32(tO(g) + lane_off + 32u * c, ov);
         }
       }
+      // pass 2: P = exp2(S scale log2e - m) chunk by chunk, written back over S
       float r8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        uint32_t raw[32], pk[16];
+        tc::tmem_ld32(tS(g) + lane_off + 32u * c, raw);
+        tc::tmem_ld_wait();
+        const bool pad = 32 * c >= kv;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
+          const float p0 = pad ? 0.f : tc::ex2(fmaf(__uint_as_float(raw[2 * e]), sl2, -m_run));
+          const float p1 = pad ? 0.f : tc::ex2(fmaf(__uint_as_float(raw[2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
           pk[e] = pack_bf16(p0, p1);
         }

@@ -62,10 +62,17 @@ struct TraceScope {
     if (g_trace) g_trace(g_trace_user, name, 1, st);
   }
 };
-#define PRISM_TRACED(NAME, ST, ...) \
-  do {                              \
-    TraceScope _ts(NAME, ST);       \
-    __VA_ARGS__;                    \
+// Launches one kernel between the trace hooks and fails the call at once if
+// the launch itself was rejected (a later successful call must not hide it).
+#define PRISM_TRACED(NAME, ST, ...)                                                     \
+  do {                                                                                  \
+    cudaGetLastError();                                                                 \
+    {                                                                                   \
+      TraceScope _ts(NAME, ST);                                                         \
+      __VA_ARGS__;                                                                      \
+    }                                                                                   \
+    const cudaError_t _le = cudaGetLastError();                                         \
+    if (_le != cudaSuccess) return prism::fail(PRISM_ECUDA, cudaGetErrorString(_le));   \
   } while (0)
 
 int fail(int code, const char *msg) {
@@ -505,7 +512,7 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
 }  // extern "C"
 
 template <int D>
-static void launch_bwd_attn(const Dims &d, dim3 grid, cudaStream_t st, const __nv_bfloat16 *Q,
+static int launch_bwd_attn(const Dims &d, dim3 grid, cudaStream_t st, const __nv_bfloat16 *Q,
                             const __nv_bfloat16 *K, const __nv_bfloat16 *Vv, const __nv_bfloat16 *dO,
                             const float *lse, const float *delta, const prism_block *blocks,
                             const int32_t *zbb, const int32_t *row_ptr, const int32_t *col,
@@ -519,6 +526,7 @@ static void launch_bwd_attn(const Dims &d, dim3 grid, cudaStream_t st, const __n
                                                       d.N, d.cap, scale, dk, dv));
   PRISM_TRACED("bsa_dq_mma_kernel", st, bsa_dq_mma_kernel<D><<<grid, 128, smem_q, st>>>(Q, K, Vv, dO, lse, delta, blocks, zbb, row_ptr, col, d.N,
                                                    d.cap, scale, dq));
+  return PRISM_OK;
 }
 
 extern "C" {
@@ -604,13 +612,14 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
     PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, kBwdThreads, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
     PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, kBwdThreads, kDqSmemBytes, st>>>(tq, tk, tv, to, a));
   } else if (d.D == 128)
-    launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
+    rc = launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
                          row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
                          static_cast<__nv_bfloat16 *>(dv));
   else
-    launch_bwd_attn<64>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
+    rc = launch_bwd_attn<64>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
                         row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
                         static_cast<__nv_bfloat16 *>(dv));
+  if (rc) return rc;
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
 }
