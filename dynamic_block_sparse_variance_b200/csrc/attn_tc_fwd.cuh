@@ -558,22 +558,24 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
       }
       tc::tc_fence_after();
       const int kv = kt.keys();
-      // pass 1: row max over the valid columns, half a row of registers at a time
+      // the whole S row in registers, one batched TMEM load
+      uint32_t raw[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tc::tmem_ld32(tS(g) + lane_off + 32u * c, raw[c]);
+      tc::tmem_ld_wait();
+      if (kv < 128) {   // a 64-key block: the upper half of the tile is padding
+#pragma unroll
+        for (int c = 2; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) raw[c][e] = __float_as_uint(-INFINITY);
+      }
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = -INFINITY;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        if (hh == 1 && kv <= 64) break;   // a 64-key block: the upper half is padding
-        uint32_t raw[2][32];
-        tc::tmem_ld32(tS(g) + lane_off + 64u * hh, raw[0]);
-        tc::tmem_ld32(tS(g) + lane_off + 64u * hh + 32u, raw[1]);
-        tc::tmem_ld_wait();
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
-      }
+        for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
       float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= sl2;
       const bool grow = mx > m_run + 8.f;
@@ -582,9 +584,25 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
         l_run *= alpha;
         m_run = mx;
       }
-      if (n > 0 && __any_sync(0xffffffffu, grow)) {
-        // S_g(n) was issued after PV_g(n-1): its completion proves O settled
+      float r8[8];
 #pragma unroll
+      for (int e = 0; e < 8; ++e) r8[e] = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
+          r8[e & 7] += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        tc::tmem_st16(tS(g) + lane_off + 16u * c, pk);
+      }
+      if (n > 0 && __any_sync(0xffffffffu, grow)) {
+        // rare: rescale O (S_g(n) was issued after PV_g(n-1), so O has settled;
+        // PV_g(n) waits for this step's P signal, issued below)
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t ov[32];
           tc::tmem_ld32(tO(g) + lane_off + 32u * c, ov);
@@ -593,25 +611,6 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
           for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
           tc::tmem_st32(tO(g) + lane_off + 32u * c, ov);
         }
-      }
-      // pass 2: P = exp2(S scale log2e - m) chunk by chunk, written back over S
-      float r8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) r8[e] = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t raw[32], pk[16];
-        tc::tmem_ld32(tS(g) + lane_off + 32u * c, raw);
-        tc::tmem_ld_wait();
-        const bool pad = 32 * c >= kv;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float p0 = pad ? 0.f : tc::ex2(fmaf(__uint_as_float(raw[2 * e]), sl2, -m_run));
-          const float p1 = pad ? 0.f : tc::ex2(fmaf(__uint_as_float(raw[2 * e + 1]), sl2, -m_run));
-          r8[e & 7] += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
-        }
-        tc::tmem_st16(tS(g) + lane_off + 16u * c, pk);
       }
       l_run += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tmem_st_wait();
