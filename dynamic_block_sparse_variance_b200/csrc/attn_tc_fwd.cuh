@@ -400,7 +400,6 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
   auto b_sfull = [&](int g) { return sBar + 8u * (9 + g); };
   auto b_pfull = [&](int g) { return sBar + 8u * (11 + g); };
   const uint32_t b_drain = sBar + 8u * 13;
-  auto b_pvd = [&](int g) { return sBar + 8u * (14 + g); };    // PV_g(n) complete
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 16);
   volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 16 + 4);
 
@@ -426,7 +425,6 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
     for (int g = 0; g < 2; ++g) {
       tc::mbar_init(b_sfull(g), 1);
       tc::mbar_init(b_pfull(g), 128);
-      tc::mbar_init(b_pvd(g), 1);
     }
     tc::mbar_init(b_drain, 1);
     *abort = 0;
@@ -523,12 +521,11 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
           }
           tc::tc_fence_after();
           issue_pv(n, g);
-          tc::mma_commit(b_pvd(g));
           if (g == 1) tc::mma_commit(b_vempty(s));
           if (n + 1 < nsteps) {
             if (g == 0 && !wait_k(n + 1)) { ok = false; break; }
-            // S_g(n+1) overwrites the columns PV_g(n) reads P from: let PV_g(n) finish first
-            if (!tc::mbar_wait(b_pvd(g), (uint32_t)n & 1u, abort, limit)) { ok = false; break; }
+            // S_g(n+1) overwrites the P columns PV_g(n) reads; the tensor pipe
+            // executes one thread's MMAs in issue order, as the other kernels rely on
             tc::tc_fence_after();
             issue_s(n + 1, g);
             if (g == 1) tc::mma_commit(b_kempty((n + 1) % kTc2Stages));
