@@ -589,11 +589,8 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          // one pair in four on the FMA pipe, the rest on the special-function unit
-          const float x0 = fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run);
-          const float x1 = fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run);
-          const float p0 = (e & 3) == 0 ? tc::ex2_poly(x0) : tc::ex2(x0);
-          const float p1 = (e & 3) == 0 ? tc::ex2_poly(x1) : tc::ex2(x1);
+          const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
           pk[e] = pack_bf16(p0, p1);
         }

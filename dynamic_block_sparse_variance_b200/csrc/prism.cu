@@ -23,14 +23,6 @@ static int g_debug_stall = 0;
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
-__global__ void exp2_selftest_kernel(const float *__restrict__ x, float *__restrict__ yp, float *__restrict__ yr,
-                                     int64_t n) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    yp[i] = tc::ex2_poly(x[i]);
-    yr[i] = exp2f(x[i]);
-  }
-}
-
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
@@ -185,15 +177,6 @@ int prism_set_option(int option, int64_t value) {
     case PRISM_OPT_DEBUG_STALL: g_debug_stall = (int)value; return PRISM_OK;
     default: return fail(PRISM_EINVAL, "unknown option");
   }
-}
-
-int prism_selftest_exp2(const float *x, float *y_poly, float *y_ref, int64_t n, prism_stream stream) {
-  if (!x || !y_poly || !y_ref || n < 0) return fail(PRISM_EINVAL, "selftest_exp2: bad argument");
-  if (n == 0) return PRISM_OK;
-  cudaStream_t st = as_stream(stream);
-  const unsigned blocks = (unsigned)std::min<int64_t>((n + 255) / 256, 65535);
-  PRISM_TRACED("exp2_selftest_kernel", st, exp2_selftest_kernel<<<blocks, 256, 0, st>>>(x, y_poly, y_ref, n));
-  return PRISM_OK;
 }
 
 int prism_set_trace(prism_trace_fn fn, void *user) {

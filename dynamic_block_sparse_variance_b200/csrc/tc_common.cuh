@@ -118,25 +118,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 0 down to -125 (inputs below are clamped there:
-// the result is then 2^-125 instead of 0, far below anything that can change a
-// softmax).  Range reduction after Cody and Waite: x = j + f with j = rint(x),
-// taken by adding 1.5 * 2^23 (round to nearest), f in [-0.5, 0.5]; 2^f by a
-// degree-3 polynomial whose coefficients were fitted here (Lawson-weighted
-// least squares on the relative error over [-0.5, 0.5], maximum relative error
-// 7.5e-5); j goes into the exponent field.  Used for part of the softmax
-// exponentials so that they do not all queue on the special-function unit.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.05517132f, f, 0.24261054f);
-  p = fmaf(p, f, 0.69326099f);
-  p = fmaf(p, f, 0.99992811f);
-  const int j = __float_as_int(t) - 0x4B400000;
-  return __int_as_float(__float_as_int(p) + (j << 23));
-}
-
 // ---- MMA -----------------------------------------------------------------------
 // Shared-memory matrix descriptor (sm_100 version 1) for a 128-byte-swizzled
 // operand: start address, leading / stride byte offsets (16-byte units).

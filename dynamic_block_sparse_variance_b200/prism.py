@@ -26,7 +26,7 @@ ENTRY_POINTS = (
     "prism_workspace_size", "prism_zone_indicator", "prism_zone_indicator_noalloc", "prism_assign_blocks",
     "prism_permute",
     "prism_unpermute", "prism_block_select", "prism_bsa_fwd", "prism_bsa_bwd",
-    "prism_selftest_exp2", "prism_set_option", "prism_set_trace", "prism_device_status", "prism_last_error",
+    "prism_set_option", "prism_set_trace", "prism_device_status", "prism_last_error",
 )
 
 TRACE_FN = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int, ctypes.c_void_p)
@@ -78,7 +78,6 @@ def lib():
             "prism_bsa_fwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, sz, _P],
             "prism_bsa_bwd": [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, i64, _P, _P, _P,
                               _P, sz, _P],
-            "prism_selftest_exp2": [_P, _P, _P, i64, _P],
             "prism_set_option": [ctypes.c_int, i64],
             "prism_set_trace": [TRACE_FN, _P],
             "prism_device_status": [_P],
@@ -165,10 +164,6 @@ def prism_bsa_bwd(p, blocks, zone_blk_base, nblk, q, k, v, o, o_res, dout, lse, 
                                _ptr(k), _ptr(v), _ptr(o), _ptr(o_res), _ptr(dout), _ptr(lse), _ptr(row_ptr),
                                _ptr(col), _ptr(nnz), col.numel(), _ptr(dq), _ptr(dk), _ptr(dv),
                                _ptr(workspace), workspace.numel(), _stream()))
-
-
-def prism_selftest_exp2(x, y_poly, y_ref):
-    _check(lib().prism_selftest_exp2(_ptr(x), _ptr(y_poly), _ptr(y_ref), x.numel(), _stream()))
 
 
 def prism_set_option(option, value):

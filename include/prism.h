@@ -248,12 +248,6 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
 #define PRISM_OPT_DEBUG_STALL 2
 int prism_set_option(int option, int64_t value);
 
-/* Diagnostic: evaluates, for n inputs x (device, float), the FMA-pipe 2^x
- * approximation the forward kernels use for part of their softmax
- * exponentials (y_poly) and CUDA's exp2f (y_ref), so that a test can bound
- * their difference.  Inputs should be <= 0 (softmax arguments). */
-int prism_selftest_exp2(const float *x, float *y_poly, float *y_ref, int64_t n, prism_stream stream);
-
 /* Kernel-launch trace hook.  When set, the library calls
  *   fn(user, kernel_name, 0, stream) just before and
  *   fn(user, kernel_name, 1, stream) just after

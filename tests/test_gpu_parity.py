@@ -266,16 +266,3 @@ def test_tc_forward_matches_warp_mma_forward():
     assert_close_attn(o0.double().numpy(), o1.double().numpy(), "O tc vs mma")
     assert float((l0 - l1).abs().max()) <= 1e-3
     assert_close_attn((o0 + r0).double().numpy(), (o1 + r1).double().numpy(), "O+residual tc vs mma")
-
-
-def test_fma_pipe_exp2_against_cuda_exp2f():
-    """The forward kernels compute a quarter of their softmax exponentials with a
-    range-reduced cubic on the FMA pipe; over the softmax range [-125, 0] it must
-    stay within 1e-4 relative of CUDA's exp2f (and of the exact value)."""
-    x = torch.cat([torch.linspace(-125.0, 0.0, 2_000_001), -torch.rand(1_000_000) * 30.0]).cuda()
-    yp, yr = torch.empty_like(x), torch.empty_like(x)
-    P.prism_selftest_exp2(x, yp, yr)
-    torch.cuda.synchronize()
-    exact = torch.exp2(x.double())
-    assert float(((yp.double() - yr.double()).abs() / yr.double()).max()) <= 1e-4
-    assert float(((yp.double() - exact).abs() / exact).max()) <= 1e-4
