@@ -109,7 +109,7 @@ def zone_indicator(V, T, H, W, audio=None, eps=EPS):
     """
     ZT, ZY, ZX = zone_grid(T, H, W)
     N = T * H * W
-    V = np.asarray(V, dtype=np.float64).reshape(N, -1)
+    V = np.asarray(V).reshape(N, -1)      # each zone is converted to float64 on its own
     Z = ZT * ZY * ZX
     sigma2_v = np.zeros((Z, 3))
     sigma2_a = np.zeros((Z, 3))
@@ -241,6 +241,19 @@ def unpermute(x_perm, perm):
     x_perm = np.asarray(x_perm)
     out = np.empty((x_perm.shape[1], x_perm.shape[0], x_perm.shape[2]), dtype=x_perm.dtype)
     out[perm] = x_perm.transpose(1, 0, 2)
+    return out
+
+
+def pool_blocks_natural(x, perm, blocks, heads=None):
+    """pool_blocks(permute(x, perm), blocks) without building the permuted copy:
+    each block's rows are gathered from the natural layout [N, heads, d].
+    Returns [len(heads), nblk, d] float64."""
+    x = np.asarray(x)
+    hs = list(range(x.shape[1])) if heads is None else list(heads)
+    out = np.empty((len(hs), len(blocks), x.shape[2]))
+    for j, (start, size, _, _) in enumerate(blocks):
+        rows = np.asarray(x[perm[start:start + size]][:, hs, :], dtype=np.float64)
+        out[:, j, :] = rows.mean(axis=0)
     return out
 
 

@@ -1,0 +1,143 @@
+"""Parity at the full benchmark grids (Small, 720p, 1080p, 2K), on sampled outputs.
+
+The GPU runs the whole path in the launch configuration bench.py times (one
+PrismSparseAttention layer over all heads).  The fp64 oracle then works from
+the same inputs on its own: the indicator and block layout of the whole grid,
+the selection of sampled query blocks (and of every query block of one head,
+for the exact selectors of sampled key blocks), and the outputs those samples
+determine: O and LSE and dQ of sampled query blocks, dK and dV of sampled key
+blocks.  Discrete results are compared exactly (selections up to near-ties);
+attention outputs within rel-RMS 1e-2 and max-abs 3e-2 beyond half a bf16 ulp.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_block_sparse_variance_b200 import prism as P
+from dynamic_block_sparse_variance_b200 import synth
+from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
+from oracle import prism_oracle as po
+from tests.helpers import assert_close_attn, selection_row_ok
+
+pytestmark = pytest.mark.gpu
+
+QUERY_SAMPLES = {"small": 6, "720p": 6, "1080p": 4, "2k": 4}
+
+
+def _head(x_cpu, h, perm):
+    """Head h of a natural-layout CPU tensor, permuted, as [1, N, d] float64."""
+    return x_cpu[:, h, :].double().numpy()[perm][None]
+
+
+@pytest.mark.parametrize("name", ["small", "720p", "1080p", "2k"])
+def test_fullsize_sampled_parity(name):
+    wl = synth.get_workload(name)
+    inp = synth.make_inputs(wl, "cuda", with_dout=wl.backward)
+    att = PrismSparseAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p)
+    att.forward(inp["q"], inp["k"], inp["v"], inp["audio"])
+    if wl.backward:
+        att.backward(inp["dout"])
+    P.prism_device_status()
+    lay = att.host_layout()
+    g_gpu, rho_gpu = att.g.cpu().numpy(), att.rho.cpu().numpy()
+    rp_gpu, cols_gpu = att.host_csr()
+    cpu = {n: (None if inp[n] is None else inp[n].cpu()) for n in inp}
+    del inp
+
+    # ---- oracle: indicator and layout of the whole grid
+    v32 = cpu["v"].float().numpy()
+    audio = cpu["audio"].double().numpy()
+    ind = po.zone_indicator(v32, wl.T, wl.H, wl.W, audio)
+    del v32
+    np.testing.assert_allclose(g_gpu, ind["g"], rtol=2e-4, atol=1e-6)
+    np.testing.assert_allclose(rho_gpu, ind["rho"], rtol=2e-4, atol=1e-6)
+    shape_id, base, blocks = po.assign_blocks(ind["g"], ind["rho"], wl.T, wl.H, wl.W)
+    np.testing.assert_array_equal(lay["shape_id"], shape_id)
+    np.testing.assert_array_equal(lay["blocks"], blocks)
+    perm = po.permutation(wl.T, wl.H, wl.W, shape_id)
+    nb = len(blocks)
+    scale = 1.0 / math.sqrt(wl.head_dim)
+    rng = np.random.default_rng(7)
+
+    # ---- sampled query blocks, stratified by block volume, random heads
+    sizes = blocks[:, 1]
+    picks = []
+    for B in (64, 128, 256):
+        cand = np.flatnonzero(sizes == B)
+        if len(cand):
+            picks += [int(c) for c in rng.choice(cand, size=min(len(cand), QUERY_SAMPLES[name] // 2 + 1), replace=False)]
+    picks = picks[:QUERY_SAMPLES[name] + 2]
+    heads = [int(h) for h in rng.integers(0, wl.heads, size=len(picks))]
+    bwd = att._bwd if wl.backward else None
+    exact = compared = 0
+    by_head = {}
+    for h, i in zip(heads, picks):
+        by_head.setdefault(h, []).append(i)
+    for h, qblocks in by_head.items():
+        q32, k32 = (cpu[n][:, h:h + 1, :].float().numpy() for n in ("q", "k"))
+        kbar = po.pool_blocks_natural(k32, perm, blocks)[0]
+        qh, kh, vh = (_head(cpu[n], h, perm) for n in ("q", "k", "v"))
+        doh = _head(cpu["dout"], h, perm) if wl.backward else None
+        for i in qblocks:
+            qbar = po.pool_blocks_natural(q32, perm, blocks[i:i + 1])[0]
+            prob = po.block_probabilities(po.block_scores(qbar, kbar, scale)[0])
+            sel_o = po.select_row(prob, wl.top_k, wl.top_p)
+            sel_g = cols_gpu[h][rp_gpu[h, i]:rp_gpu[h, i + 1]]
+            ex, ok = selection_row_ok(prob, sel_g, sel_o, wl.top_k, wl.top_p)
+            assert ok, (name, h, i)
+            exact += ex
+            if not ex:
+                continue   # a valid near-tie alternative: the outputs differ legitimately
+            compared += 1
+            row_ptr = np.zeros((1, nb + 1), dtype=np.int64)
+            row_ptr[0, i + 1:] = len(sel_o)
+            O, L = po.bsa_forward(qh, kh, vh, blocks, row_ptr, [sel_o], scale, query_blocks=[i])
+            s0, sz = blocks[i][0], blocks[i][1]
+            assert_close_attn(att.op[h, s0:s0 + sz].double().cpu().numpy(), O[0, s0:s0 + sz], f"{name} O h{h} b{i}")
+            np.testing.assert_allclose(att.lse[h, s0:s0 + sz].double().cpu().numpy(), L[0, s0:s0 + sz], atol=2e-2)
+            if wl.backward:
+                dq, _, _ = po.bsa_backward(qh, kh, vh, doh, blocks, row_ptr, [sel_o], scale, query_blocks=[i])
+                assert_close_attn(bwd["dqp"][h, s0:s0 + sz].double().cpu().numpy(), dq[0, s0:s0 + sz],
+                                  f"{name} dQ h{h} b{i}")
+    assert exact >= len(picks) - 1 and compared >= 1, f"{exact}/{len(picks)} sampled selections bit-exact"
+
+    # ---- dK, dV of sampled key blocks: the oracle selects every row of one head
+    if wl.backward:
+        h = heads[0]
+        q32, k32 = (cpu[n][:, h:h + 1, :].float().numpy() for n in ("q", "k"))
+        S = po.block_scores(po.pool_blocks_natural(q32, perm, blocks)[0],
+                            po.pool_blocks_natural(k32, perm, blocks)[0], scale)
+        rp_o = np.zeros((1, nb + 1), dtype=np.int64)
+        cols_o = []
+        sel_of_o, sel_of_g = {}, {}
+        mismatch = 0
+        for i in range(nb):
+            prob = po.block_probabilities(S[i])
+            sel_o = po.select_row(prob, wl.top_k, wl.top_p)
+            sel_g = cols_gpu[h][rp_gpu[h, i]:rp_gpu[h, i + 1]]
+            ex, ok = selection_row_ok(prob, sel_g, sel_o, wl.top_k, wl.top_p)
+            assert ok, (name, "head", h, "row", i)
+            mismatch += not ex
+            cols_o.append(sel_o)
+            rp_o[0, i + 1] = rp_o[0, i] + len(sel_o)
+            for j in sel_o:
+                sel_of_o.setdefault(int(j), []).append(i)
+            for j in sel_g:
+                sel_of_g.setdefault(int(j), []).append(i)
+        assert mismatch <= max(1, nb // 100), f"{mismatch} of {nb} rows differ at near-ties"
+        # key blocks whose selectors agree on both sides; few selectors keep the fp64 backward short
+        same = sorted((len(v), j) for j, v in sel_of_o.items() if sel_of_g.get(j) == v)
+        keys = [j for _, j in same[:2]] + [j for _, j in same[len(same) // 2: len(same) // 2 + 1]]
+        assert keys
+        qh, kh, vh, doh = (_head(cpu[n], h, perm) for n in ("q", "k", "v", "dout"))
+        cols = [np.concatenate(cols_o)]
+        for j in keys:
+            _, dk, dv = po.bsa_backward(qh, kh, vh, doh, blocks, rp_o, cols, scale, query_blocks=sel_of_o[j])
+            s0, sz = blocks[j][0], blocks[j][1]
+            assert_close_attn(bwd["dkp"][h, s0:s0 + sz].double().cpu().numpy(), dk[0, s0:s0 + sz],
+                              f"{name} dK h{h} b{j}")
+            assert_close_attn(bwd["dvp"][h, s0:s0 + sz].double().cpu().numpy(), dv[0, s0:s0 + sz],
+                              f"{name} dV h{h} b{j}")

@@ -388,3 +388,14 @@ def test_bf16_half_ulp_helper():
         b = torch.tensor(v, dtype=torch.bfloat16)
         nxt = torch.tensor(v + 2 * bf16_half_ulp(v), dtype=torch.bfloat16)
         assert float(nxt) - float(b) == 2 * bf16_half_ulp(v)
+
+
+def test_pooling_from_natural_layout_equals_pooling_of_the_permuted_copy():
+    T, H, W = 8, 16, 16
+    shape_id, base, blocks = _random_layout(T, H, W, 41)
+    perm = po.permutation(T, H, W, shape_id)
+    x = np.random.default_rng(42).standard_normal((T * H * W, 3, 4)).astype(np.float32)
+    a = po.pool_blocks(po.permute(x, perm), blocks)
+    b = po.pool_blocks_natural(x, perm, blocks)
+    np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(po.pool_blocks_natural(x, perm, blocks, heads=[2]), a[2:3], rtol=1e-12, atol=1e-12)
