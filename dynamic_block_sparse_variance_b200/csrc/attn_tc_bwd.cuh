@@ -6,8 +6,7 @@
 // bsa_dq_tc_kernel    one CTA per (128-row query tile, head), walking S_i:
 //   S_n = Q K_n^T and dP_n = dO V_n^T into tensor memory; one thread per query
 //   row turns them into dS = P (dP - D) with P = exp2(S log2e scale - LSE log2e),
-//   written over S as two bf16 parts (hi, and the rounding remainder lo);
-//   dQ += dS_hi K_n + dS_lo K_n with both read from tensor memory.
+//   written as bf16 over S; dQ += dS K_n with dS read from tensor memory.
 //   TMEM: S0 | S1 | dP | dQ (4 x 128 columns).
 //
 // bsa_dkdv_tc_kernel  one CTA per (128-key tile, head), walking the query
@@ -212,13 +211,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
         if (n + 1 < nsteps && !issue_dp(n + 1)) break;
         const int ks = n % kDqKStages;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)   // dQ += dS_hi K_n, 16 keys per step
+        for (int k = 0; k < 8; ++k)   // dQ += dS_n K_n, 16 keys per step
           tc::mma_ts(tdQ, tS(n & 1) + half_col(k), tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
                      (n > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)   // dQ += dS_lo K_n (the bf16 rounding remainder of dS)
-          tc::mma_ts(tdQ, tS(n & 1) + half_col(k) + 32u, tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024),
-                     idMN, 1u);
         tc::mma_commit(b_kempty(ks));
       }
       tc::mma_commit(b_drain);
@@ -256,22 +251,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       tc::tmem_ld_wait();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        // dS in two bf16 parts, hi = bf16(dS) and lo = bf16(dS - hi): dQ sums dS k
-        // over many keys with heavy cancellation (each row of dS sums to zero),
-        // so a single bf16 rounding of dS would dominate its error
-        uint32_t hi[16], lo[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c0 = 64 * half + 32 * cc + 2 * e;
           const float p0 = (c0 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e]), sl2, -lse2)) : 0.f;
           const float p1 = (c0 + 1 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e + 1]), sl2, -lse2)) : 0.f;
-          const float d0 = p0 * (__uint_as_float(pv[cc][2 * e]) - dl);
-          const float d1 = p1 * (__uint_as_float(pv[cc][2 * e + 1]) - dl);
-          hi[e] = pack_bf16(d0, d1);
-          lo[e] = pack_bf16(d0 - bf16_lo(hi[e]), d1 - bf16_hi(hi[e]));
+          pk[e] = pack_bf16(p0 * (__uint_as_float(pv[cc][2 * e]) - dl), p1 * (__uint_as_float(pv[cc][2 * e + 1]) - dl));
         }
-        tc::tmem_st16(tS(b) + lane_off + 64u * half + 16u * cc, hi);
-        tc::tmem_st16(tS(b) + lane_off + 64u * half + 32u + 16u * cc, lo);
+        tc::tmem_st16(tS(b) + lane_off + 64u * half + 16u * cc, pk);
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
