@@ -8,11 +8,8 @@
 //               buffers, and O += P_n V_n with P_n read from tensor memory.
 //   warps 2..5  softmax, one thread per query row (its TMEM lane): S row ->
 //               running max (log2 domain, rescaled lazily only when the max
-//               grows by more than 2^8) -> P = exp2(.) written back over S as
-//               two bf16 parts, hi and the rounding remainder lo (O += P_hi V +
-//               P_lo V keeps O accurate to ~16 bits, which the backward's row
-//               sums D = rowsum(dO o O) need) -> row sum; final normalisation,
-//               O (bf16 + residual) and LSE.
+//               grows by more than 2^8) -> P = exp2(.) as bf16 written back over
+//               S -> row sum; final normalisation, O (bf16 + residual) and LSE.
 // MMA order S_0, S_1, PV_0, S_2, PV_1, ... lets QK^T of step n+1 run while the
 // softmax of step n is computed.  Every wait is bounded; a stalled wait raises
 // a CTA-wide abort, latches PRISM_ETIMEOUT and the CTA drains and frees TMEM.
@@ -216,12 +213,9 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
         if (!tc::mbar_wait(b_vfull(s), (uint32_t)(n / kTcStages) & 1u, abort, limit)) break;
         tc::tc_fence_after();
 #pragma unroll
-        for (int k = 0; k < 8; ++k)   // O += P_hi V
+        for (int k = 0; k < 8; ++k)
           tc::mma_ts(tO, tS(n & 1) + 8u * k, tc::sw128_desc(sV(s) + 2048u * k, kTcTileBytes / 2, 1024), idO,
                      (n > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)   // O += P_lo V
-          tc::mma_ts(tO, tS(n & 1) + 64u + 8u * k, tc::sw128_desc(sV(s) + 2048u * k, kTcTileBytes / 2, 1024), idO, 1u);
         tc::mma_commit(b_vempty(s));
         tc::mma_commit(b_ofull);
       }
@@ -301,18 +295,15 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        // P as two bf16 parts (hi, and the rounding remainder lo) over S
-        uint32_t hi[16], lo[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
           const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
-          hi[e] = pack_bf16(p0, p1);
-          lo[e] = pack_bf16(p0 - bf16_lo(hi[e]), p1 - bf16_hi(hi[e]));
+          pk[e] = pack_bf16(p0, p1);
         }
-        tc::tmem_st16(tS(b) + lane_off + 16u * c, hi);
-        tc::tmem_st16(tS(b) + lane_off + 64u + 16u * c, lo);
+        tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
       }
       l_run += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tmem_st_wait();
@@ -504,12 +495,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
       auto issue_pv = [&](int n, int g) {
         const int s = n % kTc2Stages;
 #pragma unroll
-        for (int k = 0; k < 8; ++k)   // O += P_hi V
+        for (int k = 0; k < 8; ++k)
           tc::mma_ts(tO(g), tS(g) + 8u * k, tc::sw128_desc(sV(s) + 2048u * k, kTcTileBytes / 2, 1024), idO,
                      (n > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)   // O += P_lo V
-          tc::mma_ts(tO(g), tS(g) + 64u + 8u * k, tc::sw128_desc(sV(s) + 2048u * k, kTcTileBytes / 2, 1024), idO, 1u);
       };
       auto wait_k = [&](int n) {
         return tc::mbar_wait(b_kfull(n % kTc2Stages), (uint32_t)(n / kTc2Stages) & 1u, abort, limit);
@@ -598,18 +586,15 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        // P as two bf16 parts (hi, and the rounding remainder lo) over S
-        uint32_t hi[16], lo[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
           const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
-          hi[e] = pack_bf16(p0, p1);
-          lo[e] = pack_bf16(p0 - bf16_lo(hi[e]), p1 - bf16_hi(hi[e]));
+          pk[e] = pack_bf16(p0, p1);
         }
-        tc::tmem_st16(tS(g) + lane_off + 16u * c, hi);
-        tc::tmem_st16(tS(g) + lane_off + 64u + 16u * c, lo);
+        tc::tmem_st16(tS(g) + lane_off + 16u * c, pk);
       }
       if (n > 0 && __any_sync(0xffffffffu, grow)) {
         // rare: rescale O (S_g(n) was issued after PV_g(n-1), so O has settled;
