@@ -64,6 +64,8 @@ class PrismSparseAttention:
         self.ws_ind = torch.empty(max(ind, 256), dtype=torch.uint8, device=dev)
         sel_min, sel_all = P.prism_workspace_size(self.p, P.PRISM_WS_SELECT)
         self.ws_sel = torch.empty(max(sel_min, min(sel_all, select_ws_bytes)), dtype=torch.uint8, device=dev)
+        fwd_ws, _ = P.prism_workspace_size(self.p, P.PRISM_WS_FWD)
+        self.ws_fwd = torch.empty(max(fwd_ws, 256), dtype=torch.uint8, device=dev)
         self._bwd = None
 
     # -- forward ------------------------------------------------------------
@@ -84,7 +86,7 @@ class PrismSparseAttention:
 
     def attend(self):
         P.prism_bsa_fwd(self.p, self.blocks, self.zone_blk_base, self.nblk, self.qp, self.kp, self.vp,
-                        self.row_ptr, self.col, self.op, self.lse, o_res=self.op_res)
+                        self.row_ptr, self.col, self.op, self.lse, o_res=self.op_res, workspace=self.ws_fwd)
 
     def forward(self, q, k, v, audio=None, out=None):
         """Natural-layout output O [N, heads, head_dim] bf16."""

@@ -8,14 +8,17 @@
 //               buffers, and O += P_n V_n with P_n read from tensor memory.
 //   warps 2..5  softmax, one thread per query row (its TMEM lane): S row ->
 //               running max (log2 domain, rescaled lazily only when the max
-//               grows by more than 2^8) -> P = exp2(.) as bf16 written back over
+//               grows by more than 2^8) -> P = exp2(.) as fp16 written back over
 //               S -> row sum; final normalisation, O (bf16 + residual) and LSE.
+// The PV product is fp16 x fp16: V comes as fp16 scaled per head by 2^e_h
+// (see v16.cuh) and the epilogue folds 2^-e_h into 1/l.
 // MMA order S_0, S_1, PV_0, S_2, PV_1, ... lets QK^T of step n+1 run while the
 // softmax of step n is computed.  Every wait is bounded; a stalled wait raises
 // a CTA-wide abort, latches PRISM_ETIMEOUT and the CTA drains and frees TMEM.
 #pragma once
 
 #include "tc_common.cuh"
+#include "v16.cuh"
 
 namespace prism {
 
@@ -30,6 +33,7 @@ struct TcFwdArgs {
   const int32_t *col;
   int64_t N, cap;
   float scale_log2;
+  const uint32_t *vmax;   // per head: bf16 bits of max |v|; V arrives as fp16 scaled by 2^e_h
   __nv_bfloat16 *o;
   __nv_bfloat16 *o_res;
   float *lse;
@@ -189,7 +193,7 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
     if (lane == 0) {
       const int nsteps = count_key_tiles(args.col, args.blocks, e0, e1);
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idO = tc::idesc_bf16(128, 128, false, true);
+      constexpr uint32_t idO = tc::idesc_f16(128, 128, false, true);   // P (TMEM) x V, fp16
       bool ok = tc::mbar_wait(b_q, 0, abort, limit);
       auto issue_s = [&](int n) -> bool {
         const int s = n % kTcStages;
@@ -301,7 +305,7 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
           const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
           const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
+          pk[e] = pack_f16(p0, p1);
         }
         tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
       }
@@ -319,7 +323,7 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
         // the single-phase drain barrier completes after the last P V
         if (__all_sync(0xffffffffu, tc::mbar_wait(b_drain, 0, abort, limit))) {
           tc::tc_fence_after();
-          inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          inv = l_run > 0.f ? pow2f(-v16_exponent(args.vmax[h])) / l_run : 0.f;
         } else {
           ok = false;
         }
@@ -480,7 +484,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
     if (lane == 0) {
       const int nsteps = count_key_tiles(args.col, args.blocks, e0, e1);
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
-      constexpr uint32_t idO = tc::idesc_bf16(128, 128, false, true);
+      constexpr uint32_t idO = tc::idesc_f16(128, 128, false, true);   // P (TMEM) x V, fp16
       bool ok = tc::mbar_wait(b_q, 0, abort, limit);
       auto issue_s = [&](int n, int g) {
         const int s = n % kTc2Stages;
@@ -592,7 +596,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
           const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
           const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
+          pk[e] = pack_f16(p0, p1);
         }
         tc::tmem_st16(tS(g) + lane_off + 16u * c, pk);
       }
@@ -621,7 +625,7 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
       if (nsteps > 0) {
         if (__all_sync(0xffffffffu, tc::mbar_wait(b_drain, 0, abort, limit))) {
           tc::tc_fence_after();
-          inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          inv = l_run > 0.f ? pow2f(-v16_exponent(args.vmax[h])) / l_run : 0.f;
         } else {
           ok = false;
         }

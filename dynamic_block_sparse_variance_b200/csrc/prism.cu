@@ -3,6 +3,7 @@
 // headers, validates arguments on the host, lays out workspaces and launches.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <mutex>
@@ -35,16 +36,17 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D map over a [rows, 128] bf16 tensor, 64 x 128 boxes, 128-byte swizzle;
-// rows past the end read as zero.
-static bool make_tile_map(CUtensorMap *map, const void *base, uint64_t rows) {
+// 2-D map over a [rows, 128] tensor of 16-bit elements (bf16 unless stated),
+// 64 x 128 boxes, 128-byte swizzle; rows past the end read as zero.
+static bool make_tile_map(CUtensorMap *map, const void *base, uint64_t rows,
+                          CUtensorMapDataType type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {128, rows};
   cuuint64_t strides[1] = {128 * 2};
   cuuint32_t box[2] = {64, 128};
   cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+  return enc(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -153,6 +155,16 @@ struct BwdWs {
   }
 };
 
+// Forward (tensor-core path): per-head max |v| and V as scaled fp16.
+struct FwdWs {
+  size_t vmax, v16, total;
+  explicit FwdWs(const Dims &d) {
+    vmax = 0;
+    v16 = align256((size_t)d.heads * 4);
+    total = d.D == 128 ? v16 + (size_t)d.heads * d.N * 128 * 2 : 0;
+  }
+};
+
 static int launch_scan(const int32_t *cnt, int64_t R, long long *part, int64_t nchunk, int64_t capacity,
                        int32_t *row_ptr, int64_t *nnz, cudaStream_t st) {
   PRISM_TRACED("scan_partial_kernel", st, scan_partial_kernel<<<(unsigned)nchunk, kScanThreads, 0, st>>>(cnt, R, part));
@@ -218,7 +230,7 @@ int prism_workspace_size(const prism_params *p, int kind, int64_t col_capacity, 
       all = w.fixed + w.per_head * d.heads;
       break;
     }
-    case PRISM_WS_FWD: *bytes = all = 0; break;
+    case PRISM_WS_FWD: *bytes = all = FwdWs(d).total; break;
     case PRISM_WS_BWD: *bytes = all = BwdWs(d, col_capacity).total; break;
     default: return fail(PRISM_EINVAL, "unknown workspace kind");
   }
@@ -454,8 +466,6 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
                   const int32_t *nblk, const void *q, const void *k, const void *v, const int32_t *row_ptr,
                   const int32_t *col, void *o, void *o_res, float *lse, void *workspace, size_t ws_bytes,
                   prism_stream stream) {
-  (void)workspace;
-  (void)ws_bytes;
   Dims d;
   const void *tens[5] = {q, k, v, o, lse};
   int rc = check_attn(p, &d, blocks, zone_blk_base, nblk, tens, 5, row_ptr, col);
@@ -469,11 +479,26 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
   auto Ores = static_cast<__nv_bfloat16 *>(o_res);
   if (o_res && !aligned16(o_res)) return fail(PRISM_EINVAL, "attention: o_res must be 16-byte aligned");
   if (d.D == 128 && g_attn_backend == 0) {
+    const FwdWs w(d);
+    if (!workspace || ws_bytes < w.total || !aligned16(workspace))
+      return fail(PRISM_EINVAL, "forward workspace missing, misaligned or below prism_workspace_size(PRISM_WS_FWD)");
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint32_t *vmax = reinterpret_cast<uint32_t *>(ws + w.vmax);
+    void *v16 = ws + w.v16;
+    // V -> fp16 scaled by 2^e_h per head (the PV product runs fp16 x fp16)
+    const int64_t words = d.N * 16;   // 16-byte words per head
+    const unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((words + 1023) / 1024, (148 * 8 + d.heads - 1) / d.heads));
+    if (cudaMemsetAsync(vmax, 0, (size_t)d.heads * 4, st) != cudaSuccess)
+      return fail(PRISM_ECUDA, "cudaMemsetAsync failed");
+    PRISM_TRACED("head_absmax_kernel", st, head_absmax_kernel<<<dim3(gx, d.heads), 256, 0, st>>>(static_cast<const uint4 *>(v), words, vmax));
+    PRISM_TRACED("v_to_f16_kernel", st, v_to_f16_kernel<<<dim3(gx, d.heads), 256, 0, st>>>(static_cast<const uint4 *>(v), words, vmax, static_cast<uint4 *>(v16)));
     CUtensorMap tq, tk, tv;
     const uint64_t rows = (uint64_t)d.heads * d.N;
-    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows))
+    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) ||
+        !make_tile_map(&tv, v16, rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
       return fail(PRISM_ECUDA, "cuTensorMapEncodeTiled failed");
     TcFwdArgs a;
+    a.vmax = vmax;
     a.blocks = blocks;
     a.zone_blk_base = zone_blk_base;
     a.row_ptr = row_ptr;

@@ -210,6 +210,10 @@ int prism_block_select(const prism_params *p, const int32_t *nblk, const float *
  *                         to prism_bsa_bwd so that D = rowsum(dO o O) sees O to
  *                         about 16 significant bits instead of 8.
  *   lse                   out [heads, N] float
+ *   workspace             >= prism_workspace_size(PRISM_WS_FWD), 16-B aligned
+ *                         (head_dim 128: the per-head max |v| and a copy of V
+ *                         in fp16 scaled by a power of two per head, so that
+ *                         O += P V runs with P in fp16; 0 bytes for head_dim 64)
  */
 int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
                   const int32_t *nblk, const void *q, const void *k, const void *v,

@@ -43,6 +43,11 @@ def test_workspace_sizes(lib):
     cap = 8 * (64 * 96 * 160 // 512)
     assert ind > 0 and sel_min >= cap * cap * 4 and sel_all >= 24 * cap * cap * 4
     assert bwd >= 4 * 10**8
+    fwd, _ = P.prism_workspace_size(p, P.PRISM_WS_FWD)
+    N = 64 * 96 * 160
+    assert 24 * N * 128 * 2 <= fwd <= 24 * N * 128 * 2 + 4096    # fp16 copy of V, per-head maxima
+    p64 = P.make_params(8, 16, 16, 2, 64, 2, 0.9)
+    assert P.prism_workspace_size(p64, P.PRISM_WS_FWD)[0] == 0
 
 
 @pytest.mark.parametrize("bad", [dict(T=7), dict(H=0), dict(head_dim=96), dict(heads=0)])

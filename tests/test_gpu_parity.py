@@ -266,3 +266,33 @@ def test_tc_forward_matches_warp_mma_forward():
     assert_close_attn(o0.double().numpy(), o1.double().numpy(), "O tc vs mma")
     assert float((l0 - l1).abs().max()) <= 1e-3
     assert_close_attn((o0 + r0).double().numpy(), (o1 + r1).double().numpy(), "O+residual tc vs mma")
+
+
+def test_forward_v_scale_is_exact():
+    """The tensor-core forward takes V as fp16 scaled by a power of two per
+    head, chosen from the head's max |v|.  V times 2^k gives the same fp16
+    operand, so O and its residual scale by exactly 2^k and LSE is unchanged,
+    with max |v| anywhere from about 2^-57 to 2^63; a head whose V is all
+    zero gives O = 0 and a zero residual."""
+    wl, inp, ora = problem("mix16")
+    att = make_att(wl)
+    _oracle_layout_on_gpu(att, ora, inp, wl)
+    v0 = att.vp.clone()
+    att.attend()
+    P.prism_device_status()
+    o_ref, r_ref, l_ref = att.op.float().clone(), att.op_res.float().clone(), att.lse.clone()
+    assert float(o_ref.abs().max()) > 0.1
+    for k in (-60, -20, 7, 60):
+        att.vp.copy_((v0.float() * 2.0 ** k).to(torch.bfloat16))
+        att.attend()
+        P.prism_device_status()
+        assert torch.equal(att.op.float(), o_ref * 2.0 ** k), k
+        assert torch.equal(att.op_res.float(), r_ref * 2.0 ** k), k
+        assert torch.equal(att.lse, l_ref), k
+    att.vp.copy_(v0)
+    att.vp[1].zero_()
+    att.attend()
+    P.prism_device_status()
+    assert torch.equal(att.op[1].float(), torch.zeros_like(o_ref[1]))
+    assert torch.equal(att.op_res[1].float(), torch.zeros_like(r_ref[1]))
+    assert torch.equal(att.op[0].float(), o_ref[0]) and torch.equal(att.op[2].float(), o_ref[2])
