@@ -13,8 +13,9 @@
 //   blocks that selected its key block (the transposed selection):
 //   S^T = K Q_n^T and dP^T = V dO_n^T into tensor memory; one thread per key
 //   row computes P^T (written back over S^T, the A operand of dV += P^T dO_n)
-//   and dS^T (written to 128-byte-swizzled shared memory, the A operand of
-//   dK += dS^T Q_n).  TMEM: dK | dV | S^T | dP^T.
+//   and dS^T (written back over dP^T, the A operand of dK += dS^T Q_n), so
+//   both products read A from tensor memory and only B from shared memory.
+//   TMEM: dK | dV | S^T | dP^T.
 //
 // Roles, bounded waits and the abort path follow the forward kernel, with
 // eight elementwise warps instead of four: warps w and w+4 share a TMEM lane
@@ -47,10 +48,6 @@ struct TcBwdArgs {
   __nv_bfloat16 *dq, *dk, *dv;
   uint32_t wait_limit;
 };
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 
 // Tile of a zone: 128 rows (blocks of 128/256) or 64 rows (blocks of 64).
 struct ZoneTile {
@@ -305,10 +302,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
 
 // ========================================================================= dK dV
 constexpr int kKvQStages = 2;
-// K, V, dS^T, 2 x (Q, dO) tiles; 2 x (LSE*log2e, D) rows of 128 floats;
-// barriers.  The dynamic shared window starts 1024-byte aligned (no static
-// shared memory in these kernels); the kernel checks it.
-constexpr int kKvSmemBytes = kTcTileBytes * (3 + 2 * kKvQStages) + 2 * 1024 + 256;
+// K, V, 2 x (Q, dO) tiles; 2 x (LSE*log2e, D) rows of 128 floats; barriers.
+// The dynamic shared window starts 1024-byte aligned (no static shared
+// memory in these kernels); the kernel checks it.
+constexpr int kKvSmemBytes = kTcTileBytes * (2 + 2 * kKvQStages) + 2 * 1024 + 256;
 
 __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                                                              const __grid_constant__ CUtensorMap tmK,
@@ -322,10 +319,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
     if (threadIdx.x == 0) set_status(PRISM_EBOUNDS);
     return;
   }
-  const uint32_t sK = sbase, sV = sbase + kTcTileBytes, sdS = sbase + 2 * kTcTileBytes;
-  auto sQ = [&](int s) { return sbase + (uint32_t)(3 + 2 * s) * kTcTileBytes; };
-  auto sO = [&](int s) { return sbase + (uint32_t)(4 + 2 * s) * kTcTileBytes; };
-  const uint32_t sStat0 = sbase + (uint32_t)(3 + 2 * kKvQStages) * kTcTileBytes;   // [2][256] floats
+  const uint32_t sK = sbase, sV = sbase + kTcTileBytes;
+  auto sQ = [&](int s) { return sbase + (uint32_t)(2 + 2 * s) * kTcTileBytes; };
+  auto sO = [&](int s) { return sbase + (uint32_t)(3 + 2 * s) * kTcTileBytes; };
+  const uint32_t sStat0 = sbase + (uint32_t)(2 + 2 * kKvQStages) * kTcTileBytes;   // [2][256] floats
   auto sStat = [&](int s) { return sStat0 + 1024u * (uint32_t)s; };
   const uint32_t sBar = sStat0 + 2048;
   const uint32_t b_kv = sBar;
@@ -333,7 +330,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
   auto b_qempty = [&](int s) { return sBar + 8u * (3 + s); };
   auto b_st = [&](int hf) { return sBar + 8u * (5 + hf); };      // S^T, dP^T of query half hf done
   auto b_p = [&](int hf) { return sBar + 8u * (7 + hf); };       // P^T, dS^T of half hf ready (128 arrivals)
-  auto b_dsfree = [&](int hf) { return sBar + 8u * (9 + hf); };  // dK finished reading dS^T half hf
   const uint32_t b_drain = sBar + 8u * 11;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 12);
   volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 12 + 4);
@@ -355,7 +351,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
     for (int hf = 0; hf < 2; ++hf) {
       tc::mbar_init(b_st(hf), 1);
       tc::mbar_init(b_p(hf), 128);
-      tc::mbar_init(b_dsfree(hf), 1);
     }
     tc::mbar_init(b_drain, 1);
     *abort = 0;
@@ -369,7 +364,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // dK | dV | S^T half A | S^T half B | dP^T half A | dP^T half B  (halves: queries 0-63, 64-127)
+  // dK | dV | S^T half A | S^T half B | dP^T half A | dP^T half B  (halves: queries 0-63, 64-127);
+  // P^T and dS^T (bf16) overwrite the first 32 columns of their S^T and dP^T halves
   const uint32_t tdK = tmem, tdV = tmem + 128;
   auto tS = [&](int hf) { return tmem + 256u + 64u * (uint32_t)hf; };
   auto tP = [&](int hf) { return tmem + 384u + 64u * (uint32_t)hf; };
@@ -449,10 +445,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
                        idMN, (acc0 || k > 0) ? 1u : 0u);
 #pragma unroll
           for (int k = 0; k < 4; ++k)   // dK += dS^T_hf Q_hf
-            tc::mma_ss(tdK, tc::sw128_desc(sdS + (uint32_t)hf * (kTcTileBytes / 2) + 32u * k, 16, 1024),
-                       tc::sw128_desc(sQ(s) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024), idMN,
-                       (acc0 || k > 0) ? 1u : 0u);
-          tc::mma_commit(b_dsfree(hf));
+            tc::mma_ts(tdK, tP(hf) + 8u * k, tc::sw128_desc(sQ(s) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024),
+                       idMN, (acc0 || k > 0) ? 1u : 0u);
           if (hf == 1) tc::mma_commit(b_qempty(s));
           if (n + 1 < nsteps) {
             if (hf == 0 && !tc::mbar_wait(b_qfull((n + 1) % kKvQStages), (uint32_t)((n + 1) / kKvQStages) & 1u,
@@ -475,7 +469,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
     const int row = 32 * q + lane;           // key row of the tile
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
     const float sl2 = args.scale_log2;
-    uint8_t *dsrow = sgen + (sdS - sbase) + row * 128 + half * (kTcTileBytes / 2);
     KeyTiles qt;
     qt.init(args.row_idx, args.blocks, e0, e1);
     int n = 0;
@@ -490,12 +483,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
       }
       const float4 *st_l = reinterpret_cast<const float4 *>(sgen + (sStat(s) - sbase)) + 16 * half;
       const float4 *st_d = st_l + 32;
+      // S^T and dP^T of this half are in; the products that read this half's
+      // P^T and dS^T of the previous tile ran before them (the MMAs execute in order)
       if (!__all_sync(0xffffffffu, tc::mbar_wait(b_st(half), (uint32_t)n & 1u, abort, limit))) {
-        ok = false;
-        break;
-      }
-      if (n > 0 &&
-          !__all_sync(0xffffffffu, tc::mbar_wait(b_dsfree(half), (uint32_t)(n - 1) & 1u, abort, limit))) {
         ok = false;
         break;
       }
@@ -533,18 +523,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
                                     p3 * (__uint_as_float(pv[cc][4 * g + 3]) - Dv.w));
         }
         tc::tmem_st16(tS(half) + lane_off + 16u * cc, pk);
-        // dS^T row into the 128-byte-swizzled K-major tile: this half's 64
-        // columns are the half-tile `half`; columns 32cc..32cc+31 of it are
-        // 16-byte chunks 4cc..4cc+3
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = (4 * cc + u) ^ (row & 7);
-          *reinterpret_cast<uint4 *>(dsrow + chunk * 16) =
-              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-        }
+        tc::tmem_st16(tP(half) + lane_off + 16u * cc, dk);
       }
       tc::tmem_st_wait();
-      fence_proxy_async_smem();
       tc::tc_fence_before();
       tc::mbar_arrive(b_p(half));
     }
