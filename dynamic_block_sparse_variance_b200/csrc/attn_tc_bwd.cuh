@@ -12,9 +12,12 @@
 // bsa_dkdv_tc_kernel  one CTA per (128-key tile, head), walking the query
 //   blocks that selected its key block (the transposed selection):
 //   S^T = K Q_n^T and dP^T = V dO_n^T into tensor memory; one thread per key
-//   row computes P^T (written back over S^T, the A operand of dV += P^T dO_n)
-//   and dS^T (written back over dP^T, the A operand of dK += dS^T Q_n), so
-//   both products read A from tensor memory and only B from shared memory.
+//   row and query half computes P^T (written back over S^T, the A operand of
+//   dV += P^T dO_n) and then dS^T (written back over dP^T, the A operand of
+//   dK += dS^T Q_n), so both products read A from tensor memory and only B
+//   from shared memory.  The tensor pipe runs dV_n, S^T_{n+1}, dK_n,
+//   dP^T_{n+1}: P^T_{n+1} overlaps dK_n and dP^T_{n+1}, dS^T_n overlaps dV_n
+//   and S^T_{n+1}, and every product is a full 128 x 128 tile.
 //   TMEM: dK | dV | S^T | dP^T.
 //
 // Roles, bounded waits and the abort path follow the forward kernel, with
@@ -174,15 +177,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
       constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);    // B MN-major
       bool ok = tc::mbar_wait(b_q, 0, abort, limit);
+      const uint64_t dQ = tc::sw128_desc(sQ, 16, 1024), dO = tc::sw128_desc(sO, 16, 1024);
       auto issue_s = [&](int n) -> bool {   // S_n = Q K_n^T
         const int ks = n % kDqKStages;
         if (!tc::mbar_wait(b_kfull(ks), (uint32_t)(n / kDqKStages) & 1u, abort, limit)) return false;
         tc::tc_fence_after();
+        const uint64_t dK = tc::sw128_desc(sK(ks), 16, 1024);
+        const uint32_t tSn = tS(n & 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tS(n & 1), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK(ks) + off, 16, 1024), idNT,
-                     k > 0);
+          tc::mma_ss(tSn, tc::desc_adv(dQ, off), tc::desc_adv(dK, off), idNT, k > 0);
         }
         return true;
       };
@@ -190,11 +195,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
         const int vs = n % kDqVStages;
         if (!tc::mbar_wait(b_vfull(vs), (uint32_t)(n / kDqVStages) & 1u, abort, limit)) return false;
         tc::tc_fence_after();
+        const uint64_t dV = tc::sw128_desc(sV(vs), 16, 1024);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tdP, tc::sw128_desc(sO + off, 16, 1024), tc::sw128_desc(sV(vs) + off, 16, 1024), idNT,
-                     k > 0);
+          tc::mma_ss(tdP, tc::desc_adv(dO, off), tc::desc_adv(dV, off), idNT, k > 0);
         }
         tc::mma_commit(b_vempty(vs));
         tc::mma_commit(b_sd(n & 1));
@@ -206,11 +211,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
         if (!tc::mbar_wait(b_ds(n & 1), (uint32_t)(n >> 1) & 1u, abort, limit)) break;
         tc::tc_fence_after();
         if (n + 1 < nsteps && !issue_dp(n + 1)) break;
-        const int ks = n % kDqKStages;
+        const uint64_t dKmn = tc::sw128_desc(sK(n % kDqKStages), kTcTileBytes / 2, 1024);
+        const uint32_t tdSn = tS(n & 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k)   // dQ += dS_n K_n, 16 keys per step
-          tc::mma_ts(tdQ, tS(n & 1) + half_col(k), tc::sw128_desc(sK(ks) + 2048u * k, kTcTileBytes / 2, 1024), idMN,
-                     (n > 0 || k > 0) ? 1u : 0u);
+          tc::mma_ts(tdQ, tdSn + half_col(k), tc::desc_adv(dKmn, 2048u * k), idMN, (n > 0 || k > 0) ? 1u : 0u);
+        const int ks = n % kDqKStages;
         tc::mma_commit(b_kempty(ks));
       }
       tc::mma_commit(b_drain);
@@ -328,8 +334,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
   const uint32_t b_kv = sBar;
   auto b_qfull = [&](int s) { return sBar + 8u * (1 + s); };    // Q_n and dO_n landed
   auto b_qempty = [&](int s) { return sBar + 8u * (3 + s); };
-  auto b_st = [&](int hf) { return sBar + 8u * (5 + hf); };      // S^T, dP^T of query half hf done
-  auto b_p = [&](int hf) { return sBar + 8u * (7 + hf); };       // P^T, dS^T of half hf ready (128 arrivals)
+  const uint32_t b_s = sBar + 8u * 5;     // S^T_n done
+  const uint32_t b_dp = sBar + 8u * 6;    // dP^T_n done
+  const uint32_t b_p = sBar + 8u * 7;     // P^T_n written (256 arrivals)
+  const uint32_t b_ds = sBar + 8u * 8;    // dS^T_n written (256 arrivals)
   const uint32_t b_drain = sBar + 8u * 11;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 12);
   volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 12 + 4);
@@ -348,10 +356,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
       tc::mbar_init(b_qfull(s), 1);
       tc::mbar_init(b_qempty(s), 1);
     }
-    for (int hf = 0; hf < 2; ++hf) {
-      tc::mbar_init(b_st(hf), 1);
-      tc::mbar_init(b_p(hf), 128);
-    }
+    tc::mbar_init(b_s, 1);
+    tc::mbar_init(b_dp, 1);
+    tc::mbar_init(b_p, 256);
+    tc::mbar_init(b_ds, 256);
     tc::mbar_init(b_drain, 1);
     *abort = 0;
     tc::fence_barrier_init();
@@ -364,11 +372,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // dK | dV | S^T half A | S^T half B | dP^T half A | dP^T half B  (halves: queries 0-63, 64-127);
-  // P^T and dS^T (bf16) overwrite the first 32 columns of their S^T and dP^T halves
-  const uint32_t tdK = tmem, tdV = tmem + 128;
-  auto tS = [&](int hf) { return tmem + 256u + 64u * (uint32_t)hf; };
-  auto tP = [&](int hf) { return tmem + 384u + 64u * (uint32_t)hf; };
+  // dK | dV | S^T | dP^T.  P^T and dS^T (bf16) overwrite S^T and dP^T: the
+  // 64 query columns of half hf hold their bf16 pairs in the first 32.
+  const uint32_t tdK = tmem, tdV = tmem + 128, tS = tmem + 256, tDP = tmem + 384;
   const uint32_t limit = args.wait_limit;
 
   if (warp == 0) {
@@ -404,60 +410,65 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // Tensor-pipe order per query tile n: dV_n, S^T_{n+1}, dK_n, dP^T_{n+1},
+      // so that P^T_{n+1} is computed while dK_n and dP^T_{n+1} run and
+      // dS^T_n while dV_n and S^T_{n+1} run.
       const int nsteps = count_key_tiles(args.row_idx, args.blocks, e0, e1);
-      constexpr uint32_t idH = tc::idesc_bf16(128, 64, false, false);    // S^T, dP^T halves: N = 64 queries
-      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);   // dV, dK: B MN-major
+      constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);   // S^T, dP^T: both K-major
+      constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);    // dV, dK: B MN-major
       bool ok = tc::mbar_wait(b_kv, 0, abort, limit);
-      // S^T_hf = K Q_hf^T and dP^T_hf = V dO_hf^T for query half hf of tile n
-      auto issue_st = [&](int n, int hf) {
-        const int s = n % kKvQStages;
+      const uint64_t dK = tc::sw128_desc(sK, 16, 1024), dV = tc::sw128_desc(sV, 16, 1024);
+      auto issue_s = [&](int n) {   // S^T_n = K Q_n^T
+        const uint64_t dQ = tc::sw128_desc(sQ(n % kKvQStages), 16, 1024);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tS(hf), tc::sw128_desc(sK + off, 16, 1024), tc::sw128_desc(sQ(s) + 8192u * hf + off, 16, 1024),
-                     idH, k > 0);
+          tc::mma_ss(tS, tc::desc_adv(dK, off), tc::desc_adv(dQ, off), idNT, k > 0);
         }
+        tc::mma_commit(b_s);
+      };
+      auto issue_dp = [&](int n) {   // dP^T_n = V dO_n^T
+        const uint64_t dO = tc::sw128_desc(sO(n % kKvQStages), 16, 1024);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tP(hf), tc::sw128_desc(sV + off, 16, 1024), tc::sw128_desc(sO(s) + 8192u * hf + off, 16, 1024),
-                     idH, k > 0);
+          tc::mma_ss(tDP, tc::desc_adv(dV, off), tc::desc_adv(dO, off), idNT, k > 0);
         }
-        tc::mma_commit(b_st(hf));
+        tc::mma_commit(b_dp);
+      };
+      auto wait_q = [&](int n) {
+        return tc::mbar_wait(b_qfull(n % kKvQStages), (uint32_t)(n / kKvQStages) & 1u, abort, limit);
       };
       if (ok && nsteps > 0) {
-        ok = tc::mbar_wait(b_qfull(0), 0, abort, limit);
+        ok = wait_q(0);
         if (ok) {
           tc::tc_fence_after();
-          issue_st(0, 0);
-          issue_st(0, 1);
+          issue_s(0);
+          issue_dp(0);
         }
       }
       for (int n = 0; ok && n < nsteps; ++n) {
         const int s = n % kKvQStages;
-        for (int hf = 0; hf < 2 && ok; ++hf) {
-          if (!tc::mbar_wait(b_p(hf), (uint32_t)n & 1u, abort, limit)) { ok = false; break; }
+        const bool more = n + 1 < nsteps;
+        if (!tc::mbar_wait(b_p, (uint32_t)n & 1u, abort, limit)) break;
+        tc::tc_fence_after();
+        const uint64_t dOmn = tc::sw128_desc(sO(s), kTcTileBytes / 2, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)   // dV += P^T_n dO_n, 16 queries per step
+          tc::mma_ts(tdV, tS + half_col(k), tc::desc_adv(dOmn, 2048u * k), idMN, (n > 0 || k > 0) ? 1u : 0u);
+        if (more) {
+          if (!wait_q(n + 1)) break;
           tc::tc_fence_after();
-          const uint32_t acc0 = (n > 0 || hf > 0) ? 1u : 0u;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)   // dV += P^T_hf dO_hf, 16 queries per step
-            tc::mma_ts(tdV, tS(hf) + 8u * k, tc::sw128_desc(sO(s) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024),
-                       idMN, (acc0 || k > 0) ? 1u : 0u);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)   // dK += dS^T_hf Q_hf
-            tc::mma_ts(tdK, tP(hf) + 8u * k, tc::sw128_desc(sQ(s) + 8192u * hf + 2048u * k, kTcTileBytes / 2, 1024),
-                       idMN, (acc0 || k > 0) ? 1u : 0u);
-          if (hf == 1) tc::mma_commit(b_qempty(s));
-          if (n + 1 < nsteps) {
-            if (hf == 0 && !tc::mbar_wait(b_qfull((n + 1) % kKvQStages), (uint32_t)((n + 1) / kKvQStages) & 1u,
-                                          abort, limit)) {
-              ok = false;
-              break;
-            }
-            tc::tc_fence_after();
-            issue_st(n + 1, hf);
-          }
+          issue_s(n + 1);
         }
+        if (!tc::mbar_wait(b_ds, (uint32_t)n & 1u, abort, limit)) break;
+        tc::tc_fence_after();
+        const uint64_t dQmn = tc::sw128_desc(sQ(s), kTcTileBytes / 2, 1024);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)   // dK += dS^T_n Q_n
+          tc::mma_ts(tdK, tDP + half_col(k), tc::desc_adv(dQmn, 2048u * k), idMN, (n > 0 || k > 0) ? 1u : 0u);
+        tc::mma_commit(b_qempty(s));
+        if (more) issue_dp(n + 1);
       }
       tc::mma_commit(b_drain);
       volatile int no_abort = 0;
@@ -468,6 +479,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
     const int half = (warp - 2) >> 2;        // query columns [64*half, 64*half + 64)
     const int row = 32 * q + lane;           // key row of the tile
     const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+    const uint32_t colS = tS + lane_off + 64u * (uint32_t)half, colDP = tDP + lane_off + 64u * (uint32_t)half;
     const float sl2 = args.scale_log2;
     KeyTiles qt;
     qt.init(args.row_idx, args.blocks, e0, e1);
@@ -483,51 +495,70 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
       }
       const float4 *st_l = reinterpret_cast<const float4 *>(sgen + (sStat(s) - sbase)) + 16 * half;
       const float4 *st_d = st_l + 32;
-      // S^T and dP^T of this half are in; the products that read this half's
-      // P^T and dS^T of the previous tile ran before them (the MMAs execute in order)
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_st(half), (uint32_t)n & 1u, abort, limit))) {
+      // ---- P^T over S^T (dV of the previous tile, which read P^T there, ran before S^T_n)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_s, (uint32_t)n & 1u, abort, limit))) {
         ok = false;
         break;
       }
       tc::tc_fence_after();
-      uint32_t sv[2][32], pv[2][32];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        tc::tmem_ld32(tS(half) + lane_off + 32u * cc, sv[cc]);
-        tc::tmem_ld32(tP(half) + lane_off + 32u * cc, pv[cc]);
-      }
+      uint32_t pv[2][32];   // S^T, then P^T as float bits, kept for dS^T
+      tc::tmem_ld32(colS, pv[0]);
+      tc::tmem_ld32(colS + 32u, pv[1]);
       tc::tmem_ld_wait();
       const bool full = qv >= 64 * half + 64;   // no padding columns in this half
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t pk[16], dk[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int g = 0; g < 8; ++g) {   // four query columns at a time
-          float4 L = st_l[8 * cc + g], Dv = st_d[8 * cc + g];
+          float4 L = st_l[8 * cc + g];
           if (!full) {
             const int c0 = 64 * half + 32 * cc + 4 * g;
-            if (c0 + 0 >= qv) { L.x = INFINITY; Dv.x = 0.f; }
-            if (c0 + 1 >= qv) { L.y = INFINITY; Dv.y = 0.f; }
-            if (c0 + 2 >= qv) { L.z = INFINITY; Dv.z = 0.f; }
-            if (c0 + 3 >= qv) { L.w = INFINITY; Dv.w = 0.f; }
+            if (c0 + 0 >= qv) L.x = INFINITY;
+            if (c0 + 1 >= qv) L.y = INFINITY;
+            if (c0 + 2 >= qv) L.z = INFINITY;
+            if (c0 + 3 >= qv) L.w = INFINITY;
           }
-          const float p0 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 0]), sl2, -L.x));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 1]), sl2, -L.y));
-          const float p2 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 2]), sl2, -L.z));
-          const float p3 = tc::ex2(fmaf(__uint_as_float(sv[cc][4 * g + 3]), sl2, -L.w));
+          const float p0 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 0]), sl2, -L.x));
+          const float p1 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 1]), sl2, -L.y));
+          const float p2 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 2]), sl2, -L.z));
+          const float p3 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 3]), sl2, -L.w));
+          pv[cc][4 * g + 0] = __float_as_uint(p0);
+          pv[cc][4 * g + 1] = __float_as_uint(p1);
+          pv[cc][4 * g + 2] = __float_as_uint(p2);
+          pv[cc][4 * g + 3] = __float_as_uint(p3);
           pk[2 * g] = pack_bf16(p0, p1);
           pk[2 * g + 1] = pack_bf16(p2, p3);
-          dk[2 * g] = pack_bf16(p0 * (__uint_as_float(pv[cc][4 * g + 0]) - Dv.x),
-                                p1 * (__uint_as_float(pv[cc][4 * g + 1]) - Dv.y));
-          dk[2 * g + 1] = pack_bf16(p2 * (__uint_as_float(pv[cc][4 * g + 2]) - Dv.z),
-                                    p3 * (__uint_as_float(pv[cc][4 * g + 3]) - Dv.w));
         }
-        tc::tmem_st16(tS(half) + lane_off + 16u * cc, pk);
-        tc::tmem_st16(tP(half) + lane_off + 16u * cc, dk);
+        tc::tmem_st16(colS + 16u * cc, pk);
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
-      tc::mbar_arrive(b_p(half));
+      tc::mbar_arrive(b_p);
+      // ---- dS^T = P^T (dP^T - D) over dP^T (dK of the previous tile ran before dP^T_n)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_dp, (uint32_t)n & 1u, abort, limit))) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t dp[32], dk[16];
+        tc::tmem_ld32(colDP + 32u * cc, dp);   // chunk 0's stores below land on columns already read
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const float4 Dv = st_d[8 * cc + g];   // padding columns have P = 0, so dS = 0 there
+          dk[2 * g] = pack_bf16(__uint_as_float(pv[cc][4 * g + 0]) * (__uint_as_float(dp[4 * g + 0]) - Dv.x),
+                                __uint_as_float(pv[cc][4 * g + 1]) * (__uint_as_float(dp[4 * g + 1]) - Dv.y));
+          dk[2 * g + 1] = pack_bf16(__uint_as_float(pv[cc][4 * g + 2]) * (__uint_as_float(dp[4 * g + 2]) - Dv.z),
+                                    __uint_as_float(pv[cc][4 * g + 3]) * (__uint_as_float(dp[4 * g + 3]) - Dv.w));
+        }
+        tc::tmem_st16(colDP + 16u * cc, dk);
+      }
+      tc::tmem_st_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(b_ds);
     }
     if (__all_sync(0xffffffffu, ok && !*abort) && row < zt.rows) {
       bool have = n > 0;

@@ -195,15 +195,17 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = tc::idesc_f16(128, 128, false, true);   // P (TMEM) x V, fp16
       bool ok = tc::mbar_wait(b_q, 0, abort, limit);
+      const uint64_t dQ = tc::sw128_desc(sQ, 16, 1024);
       auto issue_s = [&](int n) -> bool {
         const int s = n % kTcStages;
         if (!tc::mbar_wait(b_kfull(s), (uint32_t)(n / kTcStages) & 1u, abort, limit)) return false;
         tc::tc_fence_after();
+        const uint64_t dK = tc::sw128_desc(sK(s), 16, 1024);
+        const uint32_t tSn = tS(n & 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tS(n & 1), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK(s) + off, 16, 1024), idS,
-                     k > 0);
+          tc::mma_ss(tSn, tc::desc_adv(dQ, off), tc::desc_adv(dK, off), idS, k > 0);
         }
         tc::mma_commit(b_sfull(n & 1));
         tc::mma_commit(b_kempty(s));
@@ -216,10 +218,11 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
         if (!tc::mbar_wait(b_pfull(n & 1), (uint32_t)(n >> 1) & 1u, abort, limit)) break;
         if (!tc::mbar_wait(b_vfull(s), (uint32_t)(n / kTcStages) & 1u, abort, limit)) break;
         tc::tc_fence_after();
+        const uint64_t dV = tc::sw128_desc(sV(s), kTcTileBytes / 2, 1024);
+        const uint32_t tPn = tS(n & 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc::mma_ts(tO, tS(n & 1) + 8u * k, tc::sw128_desc(sV(s) + 2048u * k, kTcTileBytes / 2, 1024), idO,
-                     (n > 0 || k > 0) ? 1u : 0u);
+          tc::mma_ts(tO, tPn + 8u * k, tc::desc_adv(dV, 2048u * k), idO, (n > 0 || k > 0) ? 1u : 0u);
         tc::mma_commit(b_vempty(s));
         tc::mma_commit(b_ofull);
       }
@@ -486,22 +489,23 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
       constexpr uint32_t idS = tc::idesc_bf16(128, 128, false, false);
       constexpr uint32_t idO = tc::idesc_f16(128, 128, false, true);   // P (TMEM) x V, fp16
       bool ok = tc::mbar_wait(b_q, 0, abort, limit);
+      const uint64_t dQ[2] = {tc::sw128_desc(sQ(0), 16, 1024), tc::sw128_desc(sQ(1), 16, 1024)};
       auto issue_s = [&](int n, int g) {
-        const int s = n % kTc2Stages;
+        const uint64_t dK = tc::sw128_desc(sK(n % kTc2Stages), 16, 1024), dQg = dQ[g];
+        const uint32_t tSg = tS(g);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tS(g), tc::sw128_desc(sQ(g) + off, 16, 1024), tc::sw128_desc(sK(s) + off, 16, 1024), idS,
-                     k > 0);
+          tc::mma_ss(tSg, tc::desc_adv(dQg, off), tc::desc_adv(dK, off), idS, k > 0);
         }
         tc::mma_commit(b_sfull(g));
       };
       auto issue_pv = [&](int n, int g) {
-        const int s = n % kTc2Stages;
+        const uint64_t dV = tc::sw128_desc(sV(n % kTc2Stages), kTcTileBytes / 2, 1024);
+        const uint32_t tOg = tO(g), tPg = tS(g);
 #pragma unroll
         for (int k = 0; k < 8; ++k)
-          tc::mma_ts(tO(g), tS(g) + 8u * k, tc::sw128_desc(sV(s) + 2048u * k, kTcTileBytes / 2, 1024), idO,
-                     (n > 0 || k > 0) ? 1u : 0u);
+          tc::mma_ts(tOg, tPg + 8u * k, tc::desc_adv(dV, 2048u * k), idO, (n > 0 || k > 0) ? 1u : 0u);
       };
       auto wait_k = [&](int n) {
         return tc::mbar_wait(b_kfull(n % kTc2Stages), (uint32_t)(n / kTc2Stages) & 1u, abort, limit);

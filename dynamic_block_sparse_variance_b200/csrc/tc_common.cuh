@@ -131,6 +131,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
   return d;
 }
 
+// The descriptor of an operand `bytes` further on (a multiple of 16).  The
+// start-address field holds address/16 in its low 14 bits; shared-memory
+// addresses stay below 256 KB, so the add never carries out of the field.
+// Issuers build one descriptor per tile and step it with constant offsets.
+__device__ __forceinline__ uint64_t desc_adv(uint64_t desc, uint32_t bytes) { return desc + (uint64_t)(bytes >> 4); }
+
 // Instruction descriptor, kind::f16: bf16 x bf16 -> f32, M x N, operand majors.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                   // D = f32
