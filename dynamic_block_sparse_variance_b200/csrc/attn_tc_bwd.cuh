@@ -5,8 +5,10 @@
 //
 // bsa_dq_tc_kernel    one CTA per (128-row query tile, head), walking S_i:
 //   S_n = Q K_n^T and dP_n = dO V_n^T into tensor memory; one thread per query
-//   row turns them into dS = P (dP - D) with P = exp2(S log2e scale - LSE log2e),
-//   written as bf16 over S; dQ += dS K_n with dS read from tensor memory.
+//   row and key half turns them into dS = P (dP - D) with
+//   P = exp2(S log2e scale - LSE log2e), written as bf16 over S; dQ += dS K_n
+//   with dS read from tensor memory.  S is double-buffered and signalled on
+//   its own, so P of tile n is computed while dP_n runs.
 //   TMEM: S0 | S1 | dP | dQ (4 x 128 columns).
 //
 // bsa_dkdv_tc_kernel  one CTA per (128-key tile, head), walking the query
@@ -93,11 +95,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   auto b_kempty = [&](int s) { return sBar + 8u * (4 + s); };   // 3
   auto b_vfull = [&](int s) { return sBar + 8u * (7 + s); };    // 2
   auto b_vempty = [&](int s) { return sBar + 8u * (9 + s); };   // 2
-  auto b_sd = [&](int b) { return sBar + 8u * (11 + b); };      // S_n and dP_n done
-  auto b_ds = [&](int b) { return sBar + 8u * (13 + b); };      // dS_n written (128 arrivals)
+  auto b_s = [&](int b) { return sBar + 8u * (11 + b); };       // S_n done (buffer n & 1)
+  auto b_ds = [&](int b) { return sBar + 8u * (13 + b); };      // dS_n written (256 arrivals)
   const uint32_t b_drain = sBar + 8u * 15;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 16);
-  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 16 + 4);
+  const uint32_t b_dp = sBar + 8u * 16;                         // dP_n done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 17);
+  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 17 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -118,9 +121,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       tc::mbar_init(b_vempty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(b_sd(b), 1);
+      tc::mbar_init(b_s(b), 1);
       tc::mbar_init(b_ds(b), 256);
     }
+    tc::mbar_init(b_dp, 1);
     tc::mbar_init(b_drain, 1);
     *abort = 0;
     tc::fence_barrier_init();
@@ -189,6 +193,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
           tc::mma_ss(tSn, tc::desc_adv(dQ, off), tc::desc_adv(dK, off), idNT, k > 0);
         }
+        tc::mma_commit(b_s(n & 1));
         return true;
       };
       auto issue_dp = [&](int n) -> bool {   // dP_n = dO V_n^T
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
           tc::mma_ss(tdP, tc::desc_adv(dO, off), tc::desc_adv(dV, off), idNT, k > 0);
         }
         tc::mma_commit(b_vempty(vs));
-        tc::mma_commit(b_sd(n & 1));
+        tc::mma_commit(b_dp);
         return true;
       };
       if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
@@ -239,30 +244,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
     bool ok = true;
     for (; kt.valid(); kt.next(), ++n) {
       const int b = n & 1;
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_sd(b), (uint32_t)(n >> 1) & 1u, abort, limit))) {
+      const uint32_t colS = tS(b) + lane_off + 64u * half;
+      // ---- P from S_n (double-buffered, so this overlaps dP_n)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_s(b), (uint32_t)(n >> 1) & 1u, abort, limit))) {
         ok = false;
         break;
       }
       tc::tc_fence_after();
       const int kv = kt.keys();
-      uint32_t sv[2][32], pv[2][32];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        tc::tmem_ld32(tS(b) + lane_off + 64u * half + 32u * cc, sv[cc]);
-        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, pv[cc]);
-      }
+      uint32_t pv[2][32];   // S, then P as float bits
+      tc::tmem_ld32(colS, pv[0]);
+      tc::tmem_ld32(colS + 32u, pv[1]);
       tc::tmem_ld_wait();
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = 64 * half + 32 * cc + 2 * e;
-          const float p0 = (c0 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e]), sl2, -lse2)) : 0.f;
-          const float p1 = (c0 + 1 < kv) ? tc::ex2(fmaf(__uint_as_float(sv[cc][2 * e + 1]), sl2, -lse2)) : 0.f;
-          pk[e] = pack_bf16(p0 * (__uint_as_float(pv[cc][2 * e]) - dl), p1 * (__uint_as_float(pv[cc][2 * e + 1]) - dl));
+        for (int e = 0; e < 32; ++e) {
+          const int c = 64 * half + 32 * cc + e;
+          pv[cc][e] = __float_as_uint((c < kv) ? tc::ex2(fmaf(__uint_as_float(pv[cc][e]), sl2, -lse2)) : 0.f);
         }
-        tc::tmem_st16(tS(b) + lane_off + 64u * half + 16u * cc, pk);
+      }
+      // ---- dS = P (dP - D) over S_n
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_dp, (uint32_t)n & 1u, abort, limit))) {
+        ok = false;
+        break;
+      }
+      tc::tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t dp[32], pk[16];
+        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, dp);
+        tc::tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = pack_bf16(__uint_as_float(pv[cc][2 * e]) * (__uint_as_float(dp[2 * e]) - dl),
+                            __uint_as_float(pv[cc][2 * e + 1]) * (__uint_as_float(dp[2 * e + 1]) - dl));
+        tc::tmem_st16(colS + 16u * cc, pk);
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
