@@ -4,12 +4,13 @@
 // are bit-reproducible:
 //
 // bsa_dq_tc_kernel    one CTA per (128-row query tile, head), walking S_i:
-//   S_n = Q K_n^T and dP_n = dO V_n^T into tensor memory; one thread per query
-//   row and key half turns them into dS = P (dP - D) with
-//   P = exp2(S log2e scale - LSE log2e), written as bf16 over S; dQ += dS K_n
-//   with dS read from tensor memory.  S is double-buffered and signalled on
-//   its own, so P of tile n is computed while dP_n runs.
-//   TMEM: S0 | S1 | dP | dQ (4 x 128 columns).
+//   Q and dO sit in tensor memory for the whole walk; S_n = Q K_n^T and
+//   dP_n = dO V_n^T read only K_n and V_n from shared memory.  One thread per
+//   query row and key half turns them into dS = P (dP - D) with
+//   P = exp2(S log2e scale - LSE log2e), written as bf16 over dP; dQ += dS K_n
+//   with dS read from tensor memory.  S is released as soon as it is read, so
+//   S_{n+1} runs while P_n and dS_n are computed.
+//   TMEM: Q | dO (64 columns each) | S | dP | dQ.
 //
 // bsa_dkdv_tc_kernel  one CTA per (128-key tile, head), walking the query
 //   blocks that selected its key block (the transposed selection):
@@ -44,6 +45,7 @@ struct TcBwdArgs {
   const int32_t *col;
   const int32_t *col_ptr;   // dkdv: transposed selection
   const int32_t *row_idx;
+  const __nv_bfloat16 *q, *dout;   // dq: permuted Q and dO rows, staged into tensor memory
   const float *lse;
   const float *delta;
   const float *lse2_pad;    // dkdv: LSE*log2e and D, padded by 128 entries
@@ -75,32 +77,34 @@ struct ZoneTile {
 };
 
 // ============================================================================ dQ
-constexpr int kDqKStages = 3, kDqVStages = 2;
-constexpr int kDqSmemBytes = kTcTileBytes * (2 + kDqKStages + kDqVStages) + 256 + 1024;
+// Q and dO of the CTA's query tile stay in tensor memory for the whole walk,
+// so S = Q K_n^T and dP = dO V_n^T read only their B operand (K_n, V_n) from
+// shared memory; dS is written over dP, which frees S as soon as P has been
+// read out of it.
+constexpr int kDqKStages = 4, kDqVStages = 3;
+constexpr int kDqSmemBytes = kTcTileBytes * (kDqKStages + kDqVStages) + 256 + 1024;
 
-__global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
-                                                           const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
-                                                           const __grid_constant__ CUtensorMap tmO,
                                                            const TcBwdArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
   uint8_t *sgen = smem_raw + (sbase - smem_u32(smem_raw));
-  const uint32_t sQ = sbase, sO = sbase + kTcTileBytes;
-  auto sK = [&](int s) { return sbase + (uint32_t)(2 + s) * kTcTileBytes; };
-  auto sV = [&](int s) { return sbase + (uint32_t)(2 + kDqKStages + s) * kTcTileBytes; };
-  const uint32_t sBar = sbase + (uint32_t)(2 + kDqKStages + kDqVStages) * kTcTileBytes;
-  const uint32_t b_q = sBar;
-  auto b_kfull = [&](int s) { return sBar + 8u * (1 + s); };    // 3
-  auto b_kempty = [&](int s) { return sBar + 8u * (4 + s); };   // 3
-  auto b_vfull = [&](int s) { return sBar + 8u * (7 + s); };    // 2
-  auto b_vempty = [&](int s) { return sBar + 8u * (9 + s); };   // 2
-  auto b_s = [&](int b) { return sBar + 8u * (11 + b); };       // S_n done (buffer n & 1)
-  auto b_ds = [&](int b) { return sBar + 8u * (13 + b); };      // dS_n written (256 arrivals)
-  const uint32_t b_drain = sBar + 8u * 15;
-  const uint32_t b_dp = sBar + 8u * 16;                         // dP_n done
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 17);
-  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 17 + 4);
+  auto sK = [&](int s) { return sbase + (uint32_t)s * kTcTileBytes; };
+  auto sV = [&](int s) { return sbase + (uint32_t)(kDqKStages + s) * kTcTileBytes; };
+  const uint32_t sBar = sbase + (uint32_t)(kDqKStages + kDqVStages) * kTcTileBytes;
+  auto b_kfull = [&](int s) { return sBar + 8u * (0 + s); };    // 4
+  auto b_kempty = [&](int s) { return sBar + 8u * (4 + s); };   // 4
+  auto b_vfull = [&](int s) { return sBar + 8u * (8 + s); };    // 3
+  auto b_vempty = [&](int s) { return sBar + 8u * (11 + s); };  // 3
+  const uint32_t b_qo = sBar + 8u * 14;      // Q, dO in tensor memory (256 arrivals)
+  const uint32_t b_s = sBar + 8u * 15;       // S_n done
+  const uint32_t b_sfree = sBar + 8u * 16;   // S_n read out (256 arrivals)
+  const uint32_t b_dp = sBar + 8u * 17;      // dP_n done
+  const uint32_t b_ds = sBar + 8u * 18;      // dS_n written over dP_n (256 arrivals)
+  const uint32_t b_drain = sBar + 8u * 19;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sgen + (sBar - sbase) + 8 * 20);
+  volatile int *abort = reinterpret_cast<volatile int *>(sgen + (sBar - sbase) + 8 * 20 + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
@@ -111,7 +115,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   const int row_base = (int)((int64_t)h * args.N);
 
   if (threadIdx.x == 0) {
-    tc::mbar_init(b_q, 1);
     for (int s = 0; s < kDqKStages; ++s) {
       tc::mbar_init(b_kfull(s), 1);
       tc::mbar_init(b_kempty(s), 1);
@@ -120,11 +123,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       tc::mbar_init(b_vfull(s), 1);
       tc::mbar_init(b_vempty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(b_s(b), 1);
-      tc::mbar_init(b_ds(b), 256);
-    }
+    tc::mbar_init(b_qo, 256);
+    tc::mbar_init(b_s, 1);
+    tc::mbar_init(b_sfree, 256);
     tc::mbar_init(b_dp, 1);
+    tc::mbar_init(b_ds, 256);
     tc::mbar_init(b_drain, 1);
     *abort = 0;
     tc::fence_barrier_init();
@@ -137,21 +140,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  auto tS = [&](int b) { return tmem + 128u * (uint32_t)b; };
-  const uint32_t tdP = tmem + 256, tdQ = tmem + 384;
+  // Q (bf16 pairs) | dO (bf16 pairs) | S | dP, then dS over it | dQ
+  const uint32_t tQ = tmem, tO = tmem + 64, tS = tmem + 128, tDP = tmem + 256, tdQ = tmem + 384;
   const uint32_t limit = args.wait_limit;
 
   if (warp == 0) {
     if (lane == 0) {
-      tc::prefetch_tmap(&tmQ);
       tc::prefetch_tmap(&tmK);
       tc::prefetch_tmap(&tmV);
-      tc::prefetch_tmap(&tmO);
-      tc::mbar_expect_tx(b_q, 2 * kTcTileBytes);
-      tc::tma_load_2d(sQ, &tmQ, 0, row_base + zt.r0, b_q);
-      tc::tma_load_2d(sQ + kTcTileBytes / 2, &tmQ, 64, row_base + zt.r0, b_q);
-      tc::tma_load_2d(sO, &tmO, 0, row_base + zt.r0, b_q);
-      tc::tma_load_2d(sO + kTcTileBytes / 2, &tmO, 64, row_base + zt.r0, b_q);
       KeyTiles kt;
       kt.init(args.col, args.blocks, e0, e1);
       int nk = 0, nv = 0;
@@ -169,7 +165,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
         ++nv;
       }
       volatile int no_abort = 0;
-      tc::mbar_wait(b_q, 0, &no_abort, limit);
       for (int k = max(0, nk - kDqKStages); k < nk; ++k)
         tc::mbar_wait(b_kfull(k % kDqKStages), (uint32_t)(k / kDqKStages) & 1u, &no_abort, limit);
       for (int k = max(0, nv - kDqVStages); k < nv; ++k)
@@ -177,26 +172,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
     }
   } else if (warp == 1) {
     if (lane == 0) {
+      // Tensor-pipe order per key tile n: S_{n+1} (as soon as S_n is read out),
+      // dQ_n (once dS_n is written), dP_{n+1}.
       const int nsteps = count_key_tiles(args.col, args.blocks, e0, e1);
       constexpr uint32_t idNT = tc::idesc_bf16(128, 128, false, false);   // both operands K-major
       constexpr uint32_t idMN = tc::idesc_bf16(128, 128, false, true);    // B MN-major
-      bool ok = tc::mbar_wait(b_q, 0, abort, limit);
-      const uint64_t dQ = tc::sw128_desc(sQ, 16, 1024), dO = tc::sw128_desc(sO, 16, 1024);
-      auto issue_s = [&](int n) -> bool {   // S_n = Q K_n^T
+      bool ok = tc::mbar_wait(b_qo, 0, abort, limit);
+      auto issue_s = [&](int n) -> bool {   // S_n = Q K_n^T, Q from tensor memory
         const int ks = n % kDqKStages;
         if (!tc::mbar_wait(b_kfull(ks), (uint32_t)(n / kDqKStages) & 1u, abort, limit)) return false;
         tc::tc_fence_after();
         const uint64_t dK = tc::sw128_desc(sK(ks), 16, 1024);
-        const uint32_t tSn = tS(n & 1);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tSn, tc::desc_adv(dQ, off), tc::desc_adv(dK, off), idNT, k > 0);
+          tc::mma_ts(tS, tQ + 8u * k, tc::desc_adv(dK, off), idNT, k > 0);
         }
-        tc::mma_commit(b_s(n & 1));
+        tc::mma_commit(b_s);
         return true;
       };
-      auto issue_dp = [&](int n) -> bool {   // dP_n = dO V_n^T
+      auto issue_dp = [&](int n) -> bool {   // dP_n = dO V_n^T, dO from tensor memory
         const int vs = n % kDqVStages;
         if (!tc::mbar_wait(b_vfull(vs), (uint32_t)(n / kDqVStages) & 1u, abort, limit)) return false;
         tc::tc_fence_after();
@@ -204,25 +199,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           const uint32_t off = (uint32_t)(k >> 2) * (kTcTileBytes / 2) + (uint32_t)(k & 3) * 32u;
-          tc::mma_ss(tdP, tc::desc_adv(dO, off), tc::desc_adv(dV, off), idNT, k > 0);
+          tc::mma_ts(tDP, tO + 8u * k, tc::desc_adv(dV, off), idNT, k > 0);
         }
         tc::mma_commit(b_vempty(vs));
         tc::mma_commit(b_dp);
         return true;
       };
-      if (ok && nsteps > 0) ok = issue_s(0) && issue_dp(0);
-      for (int n = 0; ok && n < nsteps; ++n) {
-        if (n + 1 < nsteps && !issue_s(n + 1)) break;
-        if (!tc::mbar_wait(b_ds(n & 1), (uint32_t)(n >> 1) & 1u, abort, limit)) break;
+      if (ok && nsteps > 0) {
         tc::tc_fence_after();
-        if (n + 1 < nsteps && !issue_dp(n + 1)) break;
-        const uint64_t dKmn = tc::sw128_desc(sK(n % kDqKStages), kTcTileBytes / 2, 1024);
-        const uint32_t tdSn = tS(n & 1);
+        ok = issue_s(0) && issue_dp(0);
+      }
+      for (int n = 0; ok && n < nsteps; ++n) {
+        const bool more = n + 1 < nsteps;
+        if (more) {
+          if (!tc::mbar_wait(b_sfree, (uint32_t)n & 1u, abort, limit)) break;
+          if (!issue_s(n + 1)) break;
+        }
+        if (!tc::mbar_wait(b_ds, (uint32_t)n & 1u, abort, limit)) break;
+        tc::tc_fence_after();
+        const int ks = n % kDqKStages;
+        const uint64_t dKmn = tc::sw128_desc(sK(ks), kTcTileBytes / 2, 1024);
 #pragma unroll
         for (int k = 0; k < 8; ++k)   // dQ += dS_n K_n, 16 keys per step
-          tc::mma_ts(tdQ, tdSn + half_col(k), tc::desc_adv(dKmn, 2048u * k), idMN, (n > 0 || k > 0) ? 1u : 0u);
-        const int ks = n % kDqKStages;
+          tc::mma_ts(tdQ, tDP + half_col(k), tc::desc_adv(dKmn, 2048u * k), idMN, (n > 0 || k > 0) ? 1u : 0u);
         tc::mma_commit(b_kempty(ks));
+        if (more && !issue_dp(n + 1)) break;
       }
       tc::mma_commit(b_drain);
       volatile int no_abort = 0;
@@ -238,15 +239,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
     const bool vrow = row < zt.rows;
     const float lse2 = vrow ? args.lse[grow] * kLog2e : INFINITY;   // padding rows: P = 0
     const float dl = vrow ? args.delta[grow] : 0.f;
+    // this thread's row of Q and dO, head-dim columns [64*half, 64*half + 64),
+    // into tensor memory as bf16 pairs (the A-operand layout); padding rows are zero
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      uint32_t w[32];
+      if (vrow) {
+        const uint4 *src = reinterpret_cast<const uint4 *>((which ? args.dout : args.q) + grow * 128 + 64 * half);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 x = __ldg(src + u);
+          w[4 * u] = x.x; w[4 * u + 1] = x.y; w[4 * u + 2] = x.z; w[4 * u + 3] = x.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) w[e] = 0u;
+      }
+      tc::tmem_st32((which ? tO : tQ) + lane_off + 32u * (uint32_t)half, w);
+    }
+    tc::tmem_st_wait();
+    tc::tc_fence_before();
+    tc::mbar_arrive(b_qo);
     KeyTiles kt;
     kt.init(args.col, args.blocks, e0, e1);
     int n = 0;
     bool ok = true;
+    const uint32_t colS = tS + lane_off + 64u * half, colDP = tDP + lane_off + 64u * half;
     for (; kt.valid(); kt.next(), ++n) {
-      const int b = n & 1;
-      const uint32_t colS = tS(b) + lane_off + 64u * half;
-      // ---- P from S_n (double-buffered, so this overlaps dP_n)
-      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_s(b), (uint32_t)(n >> 1) & 1u, abort, limit))) {
+      // ---- P from S_n; S is released as soon as it is read out
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(b_s, (uint32_t)n & 1u, abort, limit))) {
         ok = false;
         break;
       }
@@ -256,6 +277,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       tc::tmem_ld32(colS, pv[0]);
       tc::tmem_ld32(colS + 32u, pv[1]);
       tc::tmem_ld_wait();
+      tc::tc_fence_before();
+      tc::mbar_arrive(b_sfree);
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
@@ -264,7 +287,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
           pv[cc][e] = __float_as_uint((c < kv) ? tc::ex2(fmaf(__uint_as_float(pv[cc][e]), sl2, -lse2)) : 0.f);
         }
       }
-      // ---- dS = P (dP - D) over S_n
+      // ---- dS = P (dP - D) over dP_n (dQ of the previous tile read dS there before dP_n ran)
       if (!__all_sync(0xffffffffu, tc::mbar_wait(b_dp, (uint32_t)n & 1u, abort, limit))) {
         ok = false;
         break;
@@ -273,17 +296,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
         uint32_t dp[32], pk[16];
-        tc::tmem_ld32(tdP + lane_off + 64u * half + 32u * cc, dp);
+        tc::tmem_ld32(colDP + 32u * cc, dp);   // chunk 0's stores below land on columns already read
         tc::tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           pk[e] = pack_bf16(__uint_as_float(pv[cc][2 * e]) * (__uint_as_float(dp[2 * e]) - dl),
                             __uint_as_float(pv[cc][2 * e + 1]) * (__uint_as_float(dp[2 * e + 1]) - dl));
-        tc::tmem_st16(colS + 16u * cc, pk);
+        tc::tmem_st16(colDP + 16u * cc, pk);
       }
       tc::tmem_st_wait();
       tc::tc_fence_before();
-      tc::mbar_arrive(b_ds(b));
+      tc::mbar_arrive(b_ds);
     }
     if (__all_sync(0xffffffffu, ok && !*abort) && vrow) {
       bool have = n > 0;

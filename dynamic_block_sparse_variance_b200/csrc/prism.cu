@@ -627,6 +627,8 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
     a.cap = d.cap;
     a.scale = scale;
     a.scale_log2 = scale * kLog2e;
+    a.q = Q;
+    a.dout = dO;
     a.dq = static_cast<__nv_bfloat16 *>(dq);
     a.dk = static_cast<__nv_bfloat16 *>(dk);
     a.dv = static_cast<__nv_bfloat16 *>(dv);
@@ -635,7 +637,7 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
     cudaFuncSetAttribute(bsa_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmemBytes);
     dim3 tgrid((unsigned)(d.Z * 8), d.heads);
     PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, kBwdThreads, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
-    PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, kBwdThreads, kDqSmemBytes, st>>>(tq, tk, tv, to, a));
+    PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, kBwdThreads, kDqSmemBytes, st>>>(tk, tv, a));
   } else if (d.D == 128)
     rc = launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
                          row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),
