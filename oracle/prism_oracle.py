@@ -9,7 +9,7 @@ Source: "Prism: Dynamic Sparse Attention for Native 2K Joint Video-Audio
 Generation Model Training" (arXiv 2610.05416 reading guide), sections
 "Key ideas" and "Method" §1 (variation indicator), §2 (block volume and shape
 quantisation) and §3 (hybrid top-k / top-p attention).  Where the text leaves a
-step open, the reading taken is named inline as R1..R16; the same list is kept
+step open, the reading taken is named inline as R1..R20; the same list is kept
 with the design notes of the repository.
 
 Layouts (all numpy, float64 unless stated):
@@ -19,6 +19,7 @@ Layouts (all numpy, float64 unless stated):
   zones                 m = (zt*(H/8) + zy)*(W/8) + zx, each 8x8x8 tokens
 
 Parity status per function (pins live in tests/test_oracle_pins.py):
+  audio_norms             pinned (closed forms, scaling, a library norm)
   zone_indicator          pinned (closed forms, invariants)
   block_volume            parity unpinned: the density rho(m) is a reading (R6);
                           only its threshold rule is fixed by the pages
@@ -26,6 +27,9 @@ Parity status per function (pins live in tests/test_oracle_pins.py):
   quantise_shape          pinned (hand-derived cases, product = B, enumeration)
   permutation / pooling   pinned (bijection, box tiling, round trip)
   block_select            pinned (subset brute force, invariants)
+  top_k_from_sparsity     pinned (the README's worked ratio: 0.75 keeps 25%)
+  assign_blocks (fixed)   pinned (every zone the 4x4x4 box; equals dynamic
+                          assignment wherever that picks 4x4x4)
   bsa_forward / backward  pinned (dense attention at k = all via torch SDPA,
                           finite differences, autograd of a dense masked form)
 """
@@ -52,6 +56,21 @@ SHAPES = (
     (2, 8, 8), (4, 4, 8), (4, 8, 4), (8, 2, 8), (8, 4, 4), (8, 8, 2),              # B = 128
     (4, 8, 8), (8, 4, 8), (8, 8, 4),                                                # B = 256
 )
+
+
+def audio_norms(h):
+    """Method §1: the audio coupling input a = ||h_hat||_2 per video token.
+
+    h : [N, C], the audio-to-video cross-attention output of each video token
+    over all of its channels (heads * head_dim).  Returns [N] float64: the
+    Euclidean norm of each row (R20: the norm is taken over every channel of
+    the token, all heads together).
+    """
+    h = np.asarray(h, dtype=np.float64)
+    out = np.empty(h.shape[0])
+    for n in range(h.shape[0]):
+        out[n] = math.sqrt(float(np.dot(h[n], h[n])))
+    return out
 
 
 def zone_grid(T, H, W):
@@ -177,19 +196,29 @@ def quantise_shape(ell, B):
     raise AssertionError("unreachable")
 
 
-def assign_blocks(g, rho, T, H, W, tau128=TAU_128, tau256=TAU_256):
+def assign_blocks(g, rho, T, H, W, tau128=TAU_128, tau256=TAU_256, fixed_shape=None):
     """Method §2 end to end, plus the block table of the zone-local layout (R9).
 
     Returns (shape_id [Z] int, zone_blk_base [Z+1] int, blocks) where blocks is
     an int64 array [nblk, 4] of (start, size, zone, shape_id): block b of zone m
     starts at permuted position 512*m + b*B(m) and holds B(m) tokens.
+
+    fixed_shape: the repository README's mode with the dynamic block-shape
+    assignment switched off (``enable_ivpq_dynamic_block`` false, R19): every
+    zone takes the one canonical shape given (the README's 4x4x4 chunk is
+    index 3) and g, rho are not read.
     """
     ZT, ZY, ZX = zone_grid(T, H, W)
     Z = ZT * ZY * ZX
-    g = np.asarray(g, dtype=np.float64).reshape(Z, 3)
-    Bv = block_volume(np.asarray(rho, dtype=np.float64).reshape(Z), tau128, tau256)
-    ell = optimal_log2_edges(g, Bv)
-    shape_id = np.array([quantise_shape(ell[m], Bv[m]) for m in range(Z)], dtype=np.int64)
+    if fixed_shape is not None:
+        bT, bH, bW = SHAPES[int(fixed_shape)]
+        Bv = np.full(Z, bT * bH * bW, dtype=np.int64)
+        shape_id = np.full(Z, int(fixed_shape), dtype=np.int64)
+    else:
+        g = np.asarray(g, dtype=np.float64).reshape(Z, 3)
+        Bv = block_volume(np.asarray(rho, dtype=np.float64).reshape(Z), tau128, tau256)
+        ell = optimal_log2_edges(g, Bv)
+        shape_id = np.array([quantise_shape(ell[m], Bv[m]) for m in range(Z)], dtype=np.int64)
     per_zone = ZONE_TOKENS // Bv
     base = np.zeros(Z + 1, dtype=np.int64)
     base[1:] = np.cumsum(per_zone)
@@ -304,13 +333,28 @@ def select_row(P_row, top_k, top_p):
     return np.sort(np.array(order[:count], dtype=np.int64))
 
 
-def block_select(qbar, kbar, top_k, top_p, scale):
+def top_k_from_sparsity(sparsity, nblk):
+    """The repository README's ratio form of k (``bsa_sparsity``, R15).
+
+    A sparsity s means each query block skips the share s of the key blocks
+    (0.75 keeps a quarter), so k = ceil((1 - s) * nblk), at least 1.  s is
+    taken at float32 (the width the library's parameter has) and the product
+    is formed in float64.
+    """
+    s = float(np.float32(sparsity))
+    return max(1, int(math.ceil((1.0 - s) * nblk)))
+
+
+def block_select(qbar, kbar, top_k, top_p, scale, sparsity=None):
     """Method §3 for all heads.  qbar, kbar: [heads, nblk, d].
 
     Returns (row_ptr [heads, nblk+1], cols) as a CSR per head, cols ascending
-    within a row, plus the list of per-head probability matrices.
+    within a row, plus the list of per-head probability matrices.  With a
+    sparsity ratio, k comes from top_k_from_sparsity instead of top_k.
     """
     heads, nblk, _ = np.asarray(qbar).shape
+    if sparsity:
+        top_k = top_k_from_sparsity(sparsity, nblk)
     row_ptr = np.zeros((heads, nblk + 1), dtype=np.int64)
     cols = []
     probs = []
@@ -402,21 +446,22 @@ def bsa_backward(q, k, v, dout, blocks, row_ptr, cols, scale, query_blocks=None,
 
 
 def pipeline(Q, K, V, T, H, W, audio, top_k, top_p, scale=None, eps=EPS,
-             tau128=TAU_128, tau256=TAU_256):
+             tau128=TAU_128, tau256=TAU_256, fixed_shape=None, sparsity=None):
     """The whole forward path on natural-layout inputs, in the Method's order.
 
     Returns a dict with every intermediate: indicator dict, shape_id,
     zone_blk_base, blocks, perm, permuted q/k/v, pooled q/k, CSR, O (permuted
-    and natural) and LSE.
+    and natural) and LSE.  fixed_shape and sparsity select the README's
+    variants (see assign_blocks and top_k_from_sparsity).
     """
     d = np.asarray(Q).shape[2]
     scale = 1.0 / math.sqrt(d) if not scale else scale
     ind = zone_indicator(V, T, H, W, audio, eps)
-    shape_id, base, blocks = assign_blocks(ind["g"], ind["rho"], T, H, W, tau128, tau256)
+    shape_id, base, blocks = assign_blocks(ind["g"], ind["rho"], T, H, W, tau128, tau256, fixed_shape)
     perm = permutation(T, H, W, shape_id)
     qp, kp, vp = permute(Q, perm), permute(K, perm), permute(V, perm)
     qbar, kbar = pool_blocks(qp, blocks), pool_blocks(kp, blocks)
-    row_ptr, cols, _ = block_select(qbar, kbar, top_k, top_p, scale)
+    row_ptr, cols, _ = block_select(qbar, kbar, top_k, top_p, scale, sparsity)
     O, L = bsa_forward(qp, kp, vp, blocks, row_ptr, cols, scale)
     return dict(ind=ind, shape_id=shape_id, zone_blk_base=base, blocks=blocks, perm=perm,
                 qp=qp, kp=kp, vp=vp, qbar=qbar, kbar=kbar, row_ptr=row_ptr, cols=cols,

@@ -399,3 +399,80 @@ def test_pooling_from_natural_layout_equals_pooling_of_the_permuted_copy():
     b = po.pool_blocks_natural(x, perm, blocks)
     np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(po.pool_blocks_natural(x, perm, blocks, heads=[2]), a[2:3], rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------- audio norms and variants --
+
+def test_audio_norms_closed_forms():
+    """a = ||h||_2 per token: a 3-4-5 row gives 5, a constant row c over C channels
+    gives |c| sqrt(C), a zero row 0; scaling by alpha scales a by |alpha|, an
+    orthogonal mixing of the channels leaves a unchanged, and a random matrix
+    agrees with numpy's own vector norm."""
+    h = np.zeros((4, 16))
+    h[0, 3], h[0, 9] = 3.0, -4.0
+    h[1, :] = -0.25
+    np.testing.assert_allclose(po.audio_norms(h), [5.0, 0.25 * 4.0, 0.0, 0.0], rtol=0, atol=1e-15)
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((64, 48))
+    a = po.audio_norms(x)
+    np.testing.assert_allclose(po.audio_norms(-2.5 * x), 2.5 * a, rtol=1e-14)
+    q, _ = np.linalg.qr(rng.standard_normal((48, 48)))
+    np.testing.assert_allclose(po.audio_norms(x @ q), a, rtol=1e-12)
+    np.testing.assert_allclose(a, np.linalg.norm(x, axis=1), rtol=1e-14)
+
+
+def test_top_k_from_sparsity_follows_the_readme_ratio():
+    """The README's bsa_sparsity 0.75 means each query block attends to a quarter of
+    the key blocks: k = nblk/4 whenever 4 divides nblk; a share that is not a whole
+    block rounds up; sparsity 0 keeps every block and k never drops below 1."""
+    for nblk in (8, 240, 960, 15360):
+        assert po.top_k_from_sparsity(0.75, nblk) == nblk // 4
+        assert po.top_k_from_sparsity(0.5, nblk) == nblk // 2
+        assert po.top_k_from_sparsity(0.0, nblk) == nblk
+    assert po.top_k_from_sparsity(0.75, 9) == 3            # 2.25 -> 3
+    assert po.top_k_from_sparsity(0.999, 10) == 1          # 0.01 -> 1
+    assert po.top_k_from_sparsity(1.0, 10) == 1            # never empty
+    # float32 parameter width: 0.93 is 0.93000000715..., so 960 * 0.06999999285 = 67.2 -> 68
+    assert po.top_k_from_sparsity(0.93, 960) == 68
+
+
+def test_select_with_sparsity_ratio_equals_select_with_its_k():
+    rng = np.random.default_rng(3)
+    qb, kb = rng.standard_normal((2, 12, 8)), rng.standard_normal((2, 12, 8))
+    k = po.top_k_from_sparsity(0.75, 12)
+    a = po.block_select(qb, kb, 1, 0.5, 0.4, sparsity=0.75)
+    b = po.block_select(qb, kb, k, 0.5, 0.4)
+    np.testing.assert_array_equal(a[0], b[0])
+    for x, y in zip(a[1], b[1]):
+        np.testing.assert_array_equal(x, y)
+    assert all(np.diff(a[0][h]).min() >= k for h in range(2))
+
+
+def test_fixed_shape_mode_is_the_uniform_444_tiling():
+    """enable_ivpq_dynamic_block off: every zone is cut into eight 4x4x4 boxes, in
+    raster order, whatever g and rho are; on zones where the dynamic rule itself
+    lands on 4x4x4 (isotropic g, rho >= tau_128) the two layouts coincide."""
+    T, H, W = 16, 8, 16
+    Z = (T // 8) * (H // 8) * (W // 8)
+    rng = np.random.default_rng(11)
+    g = rng.uniform(1e-4, 1.0, (Z, 3))
+    rho = rng.uniform(0, 1, Z)
+    sid, base, blocks = po.assign_blocks(g, rho, T, H, W, fixed_shape=3)
+    assert (sid == 3).all() and po.SHAPES[3] == (4, 4, 4)
+    np.testing.assert_array_equal(base, 8 * np.arange(Z + 1))
+    assert (blocks[:, 1] == 64).all()
+    np.testing.assert_array_equal(blocks[:, 0], 64 * np.arange(8 * Z))
+    perm = po.permutation(T, H, W, sid)
+    for b in range(8 * Z):
+        n = perm[64 * b: 64 * b + 64]
+        t, y, x = n // (H * W), (n // W) % H, n % W
+        for c in (t, y, x):
+            assert c.max() - c.min() == 3 and c.min() % 4 == 0
+    iso = np.full((Z, 3), 0.3)
+    dyn = po.assign_blocks(iso, np.full(Z, 0.9), T, H, W)
+    fix = po.assign_blocks(iso, np.full(Z, 0.9), T, H, W, fixed_shape=3)
+    for u, v in zip(dyn, fix):
+        np.testing.assert_array_equal(u, v)
+    # other fixed shapes keep their own volume
+    sid, base, blocks = po.assign_blocks(None, None, T, H, W, fixed_shape=13)
+    assert (blocks[:, 1] == 256).all() and (np.diff(base) == 2).all()
