@@ -25,12 +25,17 @@ class PrismSparseAttention:
     quarter of them on large ones.  With ``training`` the forward also keeps
     the bf16 rounding residual of O for the backward's row sums.
     ``select_ws_bytes`` bounds the block-score workspace (heads are processed
-    in passes that fit).
+    in passes that fit).  The Prism README's variants: ``fixed_shape`` (0 =
+    dynamic shapes; ``P.PRISM_FIXED_444`` = every zone in 4x4x4 blocks, and the
+    indicator is skipped) and ``sparsity`` (k from the ratio instead of top_k).
     """
 
     def __init__(self, T, H, W, heads, head_dim, top_k, top_p, *, tau128=0.5, tau256=0.25, eps=1e-4,
-                 scale=0.0, col_capacity=None, select_ws_bytes=4 << 30, training=True, device="cuda"):
-        self.p = P.make_params(T, H, W, heads, head_dim, top_k, top_p, tau128, tau256, eps, scale)
+                 scale=0.0, col_capacity=None, select_ws_bytes=4 << 30, training=True, device="cuda",
+                 fixed_shape=P.PRISM_DYNAMIC_SHAPES, sparsity=0.0):
+        self.p = P.make_params(T, H, W, heads, head_dim, top_k, top_p, tau128, tau256, eps, scale,
+                               fixed_shape, sparsity)
+        self.fixed_shape = fixed_shape
         self.T, self.H, self.W, self.heads, self.D = T, H, W, heads, head_dim
         self.N = T * H * W
         self.Z = self.N // 512
@@ -90,7 +95,8 @@ class PrismSparseAttention:
 
     def forward(self, q, k, v, audio=None, out=None):
         """Natural-layout output O [N, heads, head_dim] bf16."""
-        self.indicator(v, audio)
+        if self.fixed_shape == P.PRISM_DYNAMIC_SHAPES:
+            self.indicator(v, audio)
         self.assign()
         self.permute(q, k, v)
         self.select()

@@ -247,9 +247,10 @@ __device__ __forceinline__ int quantise_shape(const double ell[3], int B) {
   return first;
 }
 
+// fixed > 0: every zone takes canonical shape fixed - 1 (g and rho unread).
 __global__ void __launch_bounds__(1024) assign_blocks_kernel(const float *__restrict__ g,
                                                              const float *__restrict__ rho, int Z,
-                                                             float tau128, float tau256,
+                                                             float tau128, float tau256, int fixed,
                                                              uint8_t *__restrict__ shape_id,
                                                              int32_t *__restrict__ zone_blk_base,
                                                              prism_block *__restrict__ blocks,
@@ -262,7 +263,11 @@ __global__ void __launch_bounds__(1024) assign_blocks_kernel(const float *__rest
   for (int m0 = 0; m0 < Z; m0 += blockDim.x) {
     const int m = m0 + threadIdx.x;
     int sid = 0, B = 0, nb = 0;
-    if (m < Z) {
+    if (m < Z && fixed > 0) {
+      sid = fixed - 1;
+      B = shape_volume(sid);
+      nb = kZoneTokens / B;
+    } else if (m < Z) {
       const float r = rho[m];
       B = r >= tau128 ? 64 : (r >= tau256 ? 128 : 256);
       const double S = log2((double)B);

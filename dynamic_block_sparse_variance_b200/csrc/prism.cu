@@ -12,6 +12,7 @@
 #include "attn_mma_bwd.cuh"
 #include "attn_tc_bwd.cuh"
 #include "indicator.cuh"
+#include "norms.cuh"
 #include "permute.cuh"
 #include "select.cuh"
 
@@ -100,6 +101,8 @@ static int check_params(const prism_params *p, Dims *d) {
   d->cap = d->Z * kMaxBlocksPerZone;
   d->C = (int64_t)p->heads * p->head_dim;
   if (d->Z > 65535) return fail(PRISM_EINVAL, "grid has more than 65535 macro-zones");
+  if (p->fixed_shape < 0 || p->fixed_shape > 16) return fail(PRISM_EINVAL, "fixed_shape must be 0 or 1..16");
+  if (!(p->sparsity >= 0.f && p->sparsity <= 1.f)) return fail(PRISM_EINVAL, "sparsity must be in [0, 1]");
   return PRISM_OK;
 }
 
@@ -238,6 +241,27 @@ int prism_workspace_size(const prism_params *p, int kind, int64_t col_capacity, 
   return PRISM_OK;
 }
 
+int prism_audio_norms(const void *h, int h_dtype, int64_t N, int C, float *a, prism_stream stream) {
+  if (N < 0 || C <= 0) return fail(PRISM_EINVAL, "audio_norms: N must be >= 0 and C > 0");
+  if (h_dtype != PRISM_BF16 && h_dtype != PRISM_F32) return fail(PRISM_EINVAL, "audio_norms: dtype must be bf16 or f32");
+  if (C % (h_dtype == PRISM_BF16 ? 8 : 4)) return fail(PRISM_EINVAL, "audio_norms: C must fill whole 16-byte vectors");
+  if (N == 0) return PRISM_OK;
+  if (!h || !a) return fail(PRISM_EINVAL, "audio_norms: NULL argument");
+  if (!aligned16(h)) return fail(PRISM_EINVAL, "audio_norms: h must be 16-byte aligned");
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t rows_per_block = kNormThreads / 32;
+  const unsigned grid = (unsigned)std::min<int64_t>((N + rows_per_block - 1) / rows_per_block, (int64_t)sms * 8);
+  cudaStream_t st = as_stream(stream);
+  if (h_dtype == PRISM_BF16)
+    PRISM_TRACED("audio_norms_kernel", st, audio_norms_kernel<__nv_bfloat16><<<grid, kNormThreads, 0, st>>>(
+                                               static_cast<const __nv_bfloat16 *>(h), N, C, a));
+  else
+    PRISM_TRACED("audio_norms_kernel", st, audio_norms_kernel<float><<<grid, kNormThreads, 0, st>>>(
+                                               static_cast<const float *>(h), N, C, a));
+  return PRISM_OK;
+}
+
 int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, const float *audio, float *g,
                          float *rho, float *debug, void *workspace, size_t ws_bytes, prism_stream stream) {
   Dims d;
@@ -340,9 +364,9 @@ int prism_assign_blocks(const prism_params *p, const float *g, const float *rho,
   Dims d;
   int rc = check_params(p, &d);
   if (rc) return rc;
-  if (!g || !rho || !shape_id || !zone_blk_base || !blocks || !nblk)
+  if ((p->fixed_shape == PRISM_DYNAMIC_SHAPES && (!g || !rho)) || !shape_id || !zone_blk_base || !blocks || !nblk)
     return fail(PRISM_EINVAL, "assign_blocks: NULL argument");
-  PRISM_TRACED("assign_blocks_kernel", as_stream(stream), assign_blocks_kernel<<<1, 1024, 0, as_stream(stream)>>>(g, rho, (int)d.Z, p->tau128, p->tau256, shape_id,
+  PRISM_TRACED("assign_blocks_kernel", as_stream(stream), assign_blocks_kernel<<<1, 1024, 0, as_stream(stream)>>>(g, rho, (int)d.Z, p->tau128, p->tau256, p->fixed_shape, shape_id,
                                                           zone_blk_base, blocks, nblk));
   PRISM_CUDA_CHECK_LAUNCH();
   return PRISM_OK;
@@ -407,7 +431,7 @@ int prism_block_select(const prism_params *p, const int32_t *nblk, const float *
   if (!nblk || !q_pooled || !k_pooled || !row_ptr || !nnz || (!col && col_capacity > 0))
     return fail(PRISM_EINVAL, "block_select: NULL argument");
   if (!aligned16(q_pooled) || !aligned16(k_pooled)) return fail(PRISM_EINVAL, "block_select: pooled must be 16-byte aligned");
-  if (p->top_k < 1) return fail(PRISM_EINVAL, "top_k must be >= 1");
+  if (p->sparsity == 0.f && p->top_k < 1) return fail(PRISM_EINVAL, "top_k must be >= 1");
   if (!(p->top_p > 0.f && p->top_p <= 1.f)) return fail(PRISM_EINVAL, "top_p must be in (0, 1]");
   const size_t key_bytes = (size_t)d.cap * 4;
   if (key_bytes + sizeof(SelShared) > 227 * 1024) return fail(PRISM_EINVAL, "too many blocks per head for selection");
@@ -429,7 +453,7 @@ int prism_block_select(const prism_params *p, const int32_t *nblk, const float *
     const int nh = std::min(hp, d.heads - h0);
     PRISM_TRACED("block_scores_kernel", st, block_scores_kernel<<<dim3(tiles, tiles, nh), 256, 0, st>>>(q_pooled, k_pooled, d.D, d.cap, nblk, h0, scale, S));
     PRISM_TRACED("row_cut_kernel", st, row_cut_kernel<<<dim3((unsigned)d.cap, nh), kSelThreads, key_bytes, st>>>(S, d.cap, nblk, h0, p->top_k,
-                                                                               p->top_p, cnt, ckey, cq));
+                                                                               p->sparsity, p->top_p, cnt, ckey, cq));
   }
   PRISM_CUDA_CHECK_LAUNCH();
   rc = launch_scan(cnt, w.R, part, w.nchunk, col_capacity, row_ptr, nnz, st);

@@ -131,7 +131,7 @@ struct SelShared {
 
 __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__restrict__ S, int64_t cap,
                                                              const int32_t *__restrict__ nblk_p, int h0,
-                                                             int top_k, float top_p,
+                                                             int top_k, float sparsity, float top_p,
                                                              int32_t *__restrict__ cnt,
                                                              uint32_t *__restrict__ cut_key,
                                                              int32_t *__restrict__ cut_q) {
@@ -164,7 +164,9 @@ __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__res
   for (int j = threadIdx.x; j < n; j += kSelThreads) tot += block_mass(key_score(keys[j]), smax, invZ);
   tot = sel_reduce(tot, sh.ured, [](unsigned long long a, unsigned long long b) { return a + b; });
   const unsigned long long pf = __double2ull_rn((double)top_p * kMassOne);
-  const unsigned long long kk = (unsigned long long)min(top_k, n);
+  // k: absolute, or the ratio form ceil((1 - sparsity) * nblk), at least 1
+  const int k_eff = sparsity > 0.f ? max(1, (int)ceil((1.0 - (double)sparsity) * (double)n)) : top_k;
+  const unsigned long long kk = (unsigned long long)min(k_eff, n);
   if (tot < pf) {  // top-p never reached: the whole row
     if (threadIdx.x == 0) {
       cnt[row] = n;

@@ -23,7 +23,7 @@ PRISM_OPT_ATTN_BACKEND, PRISM_OPT_WAIT_LIMIT, PRISM_OPT_DEBUG_STALL = 0, 1, 2
 
 # Entry points declared in include/prism.h, in declaration order.
 ENTRY_POINTS = (
-    "prism_workspace_size", "prism_zone_indicator", "prism_zone_indicator_noalloc", "prism_assign_blocks",
+    "prism_workspace_size", "prism_audio_norms", "prism_zone_indicator", "prism_zone_indicator_noalloc", "prism_assign_blocks",
     "prism_permute",
     "prism_unpermute", "prism_block_select", "prism_bsa_fwd", "prism_bsa_bwd",
     "prism_set_option", "prism_set_trace", "prism_device_status", "prism_last_error",
@@ -42,7 +42,8 @@ class prism_params(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("W", ctypes.c_int32),
                 ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("tau128", ctypes.c_float), ("tau256", ctypes.c_float), ("eps", ctypes.c_float),
-                ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float), ("scale", ctypes.c_float)]
+                ("top_k", ctypes.c_int32), ("top_p", ctypes.c_float), ("scale", ctypes.c_float),
+                ("fixed_shape", ctypes.c_int32), ("sparsity", ctypes.c_float)]
 
 
 class prism_block(ctypes.Structure):
@@ -50,8 +51,15 @@ class prism_block(ctypes.Structure):
                 ("shape", ctypes.c_int32)]
 
 
-def make_params(T, H, W, heads, head_dim, top_k, top_p, tau128=0.5, tau256=0.25, eps=1e-4, scale=0.0):
-    return prism_params(T, H, W, heads, head_dim, tau128, tau256, eps, top_k, top_p, scale)
+PRISM_DYNAMIC_SHAPES = 0
+PRISM_FIXED_444 = 3 + 1      # PRISM_FIXED_SHAPE(3): the 4x4x4 box
+
+
+def make_params(T, H, W, heads, head_dim, top_k, top_p, tau128=0.5, tau256=0.25, eps=1e-4, scale=0.0,
+                fixed_shape=PRISM_DYNAMIC_SHAPES, sparsity=0.0):
+    """fixed_shape: 0 = dynamic shapes, s + 1 = canonical shape s everywhere;
+    sparsity: 0 = absolute top_k, else k = max(1, ceil((1 - sparsity) * nblk))."""
+    return prism_params(T, H, W, heads, head_dim, tau128, tau256, eps, top_k, top_p, scale, fixed_shape, sparsity)
 
 
 _lib = None
@@ -69,6 +77,7 @@ def lib():
         i64, sz, pp = ctypes.c_int64, ctypes.c_size_t, ctypes.POINTER(prism_params)
         sig = {
             "prism_workspace_size": [pp, ctypes.c_int, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)],
+            "prism_audio_norms": [_P, ctypes.c_int, i64, ctypes.c_int, _P, _P],
             "prism_zone_indicator": [pp, _P, ctypes.c_int, _P, _P, _P, _P, _P, sz, _P],
             "prism_zone_indicator_noalloc": [pp, _P, ctypes.c_int, _P, _P, _P, _P, _P],
             "prism_assign_blocks": [pp, _P, _P, _P, _P, _P, _P, _P],
@@ -118,6 +127,12 @@ def prism_workspace_size(p, kind, col_capacity=0):
     a, b = ctypes.c_size_t(0), ctypes.c_size_t(0)
     _check(lib().prism_workspace_size(ctypes.byref(p), kind, col_capacity, ctypes.byref(a), ctypes.byref(b)))
     return a.value, b.value
+
+
+def prism_audio_norms(h, a):
+    """a[n] = ||h[n, :]||_2 for a row-major [N, C] tensor h (bf16 or f32)."""
+    _check(lib().prism_audio_norms(_ptr(h), _dtype(h), h.shape[0], h.shape[1] if h.dim() > 1 else 0, _ptr(a),
+                                   _stream()))
 
 
 def prism_zone_indicator(p, V, audio, g, rho, debug, workspace):

@@ -73,6 +73,17 @@ typedef void *prism_stream; /* cudaStream_t */
  *   top_p     cumulative probability mass to keep (Method §3), in (0, 1].
  *   scale     softmax scale for block scores and attention; 0 means
  *             1/sqrt(head_dim).
+ * The two variants of the Prism repository's configuration table (its README):
+ *   fixed_shape  PRISM_DYNAMIC_SHAPES (0): the dynamic assignment of Method §2.
+ *             PRISM_FIXED_SHAPE(s) (s + 1, s a canonical shape index 0..15):
+ *             every zone takes shape s and g, rho are not read.  With the
+ *             dynamic assignment switched off (enable_ivpq_dynamic_block
+ *             false) the README's blocks are 4x4x4: PRISM_FIXED_444.
+ *   sparsity  0: k = top_k.  In (0, 1]: the README's ratio form bsa_sparsity,
+ *             the share of key blocks a query block skips, so
+ *             k = max(1, ceil((1 - sparsity) * nblk)) (formed in double from
+ *             this float) and top_k is not read.
+ * A zero-initialised tail (both 0) gives the method as the paper states it.
  */
 typedef struct {
   int32_t T, H, W;
@@ -82,7 +93,13 @@ typedef struct {
   int32_t top_k;
   float top_p;
   float scale;
+  int32_t fixed_shape;
+  float sparsity;
 } prism_params;
+
+#define PRISM_DYNAMIC_SHAPES 0
+#define PRISM_FIXED_SHAPE(s) ((s) + 1)
+#define PRISM_FIXED_444 PRISM_FIXED_SHAPE(3)
 
 /* One block of the zone-local layout: permuted rows [start, start+size) of
  * every head, inside zone `zone`, of canonical shape index `shape`. */
@@ -96,6 +113,18 @@ typedef struct {
  * col_capacity matters for PRISM_WS_BWD only.  Host-only; returns a status. */
 int prism_workspace_size(const prism_params *p, int kind, int64_t col_capacity,
                          size_t *bytes, size_t *bytes_all_heads);
+
+/*
+ * Method §1, the indicator's audio input: a_n = ||h_n||_2, the Euclidean norm
+ * of each video token's audio-to-video cross-attention output over all of its
+ * channels (heads * head_dim of that layer, all heads together).  The pages
+ * cache these norms from the preceding layer; this is the producer.
+ *   h      [N, C] row-major, PRISM_BF16 or PRISM_F32, 16-byte aligned; C > 0 a
+ *          multiple of 8 (bf16) or 4 (f32).  Squares are summed in float.
+ *   a      out [N] float.
+ * N = 0 launches nothing.  Host-detected errors return PRISM_EINVAL.
+ */
+int prism_audio_norms(const void *h, int h_dtype, int64_t N, int C, float *a, prism_stream stream);
 
 /*
  * Method §1 and the density of §2: per macro-zone m, the directional video
@@ -148,7 +177,9 @@ int prism_zone_indicator_noalloc(const prism_params *p, const void *V, int v_dty
  * log2 g), and the nearest of the 16 candidate shapes (edges in {2,4,8},
  * product B; canonical order volume then (bT,bH,bW) ascending; distance ties
  * within 1e-9 go to the lowest index).  Decisions are taken in double.
- *   g [Z,3], rho [Z]        in (as produced by prism_zone_indicator)
+ *   g [Z,3], rho [Z]        in (as produced by prism_zone_indicator); not
+ *                           read, and may be NULL, when p->fixed_shape names a
+ *                           fixed shape
  *   shape_id [Z]            out, canonical shape index
  *   zone_blk_base [Z+1]     out, first block of each zone (exclusive scan)
  *   blocks [8Z]             out, block table in zone-local order
@@ -182,7 +213,9 @@ int prism_unpermute(const prism_params *p, const uint8_t *shape_id, const void *
  * S_i = Top-k(P_i, k) U Top-p(P_i, p): key blocks ranked by (score
  * descending, index ascending); S_i is the longest of the first min(k, nblk)
  * and the shortest prefix whose mass reaches p (mass summed in 2^-40 fixed
- * point).  Output is a CSR per head over rows h*8Z + i, columns ascending.
+ * point).  k is p->top_k, or comes from p->sparsity and nblk on the device
+ * when that is set.  Output is a CSR per head over rows h*8Z + i, columns
+ * ascending.
  *   nblk [1]              in (device), from prism_assign_blocks
  *   q_pooled, k_pooled    in [heads, 8Z, head_dim] float
  *   row_ptr               out [heads*8Z + 1] int32 (rows i >= nblk are empty)

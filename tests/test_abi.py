@@ -72,3 +72,36 @@ def test_null_and_misaligned_pointers_rejected(lib):
     bad_p = P.make_params(8, 16, 16, 2, 64, 0, 0.9)
     assert lib.prism_block_select(ctypes.byref(bad_p), fake, fake, fake, fake, fake, 0, fake, fake, 1 << 30,
                                   None) == P.PRISM_EINVAL
+
+
+@pytest.mark.parametrize("bad", [dict(fixed_shape=-1), dict(fixed_shape=17), dict(sparsity=-0.1),
+                                 dict(sparsity=1.5), dict(sparsity=float("nan"))])
+def test_variant_params_rejected_on_host(lib, bad):
+    kw = dict(T=8, H=16, W=16, heads=2, head_dim=64, top_k=2, top_p=0.9)
+    kw.update(bad)
+    with pytest.raises(P.PrismError) as e:
+        P.prism_workspace_size(P.make_params(**kw), P.PRISM_WS_INDICATOR)
+    assert e.value.code == P.PRISM_EINVAL
+
+
+def test_variant_params_accepted(lib):
+    for kw in (dict(fixed_shape=P.PRISM_FIXED_444), dict(fixed_shape=16), dict(sparsity=0.75),
+               dict(sparsity=1.0, top_k=0)):
+        p = P.make_params(8, 16, 16, 2, 64, kw.pop("top_k", 2), 0.9, **kw)
+        assert P.prism_workspace_size(p, P.PRISM_WS_SELECT)[0] > 0
+    # dynamic shapes need g and rho; a fixed shape does not read them
+    p = P.make_params(8, 16, 16, 2, 64, 2, 0.9)
+    assert lib.prism_assign_blocks(ctypes.byref(p), None, None, None, None, None, None, None) == P.PRISM_EINVAL
+    assert b"NULL" in lib.prism_last_error()
+
+
+def test_audio_norms_host_checks(lib):
+    fake = ctypes.c_void_p(0x1000)
+    assert lib.prism_audio_norms(fake, P.PRISM_BF16, 10, 12, fake, None) == P.PRISM_EINVAL    # C % 8
+    assert lib.prism_audio_norms(fake, P.PRISM_F32, 10, 6, fake, None) == P.PRISM_EINVAL      # C % 4
+    assert lib.prism_audio_norms(fake, 7, 10, 8, fake, None) == P.PRISM_EINVAL                # dtype
+    assert lib.prism_audio_norms(ctypes.c_void_p(0x1008), P.PRISM_BF16, 10, 8, fake, None) == P.PRISM_EINVAL
+    assert b"aligned" in lib.prism_last_error()
+    assert lib.prism_audio_norms(None, P.PRISM_BF16, 10, 8, fake, None) == P.PRISM_EINVAL
+    assert lib.prism_audio_norms(fake, P.PRISM_BF16, -1, 8, fake, None) == P.PRISM_EINVAL
+    assert lib.prism_audio_norms(None, P.PRISM_BF16, 0, 8, None, None) == P.PRISM_OK          # empty: no launch
