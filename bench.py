@@ -128,6 +128,33 @@ def executed_pairs(att):
 KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_fwd_tc_kernel": 4, "bsa_fwd_tc2_kernel": 4, "bsa_dkdv_mma_kernel": 8,
                      "bsa_dkdv_tc_kernel": 8, "bsa_dq_mma_kernel": 2, "bsa_dq_tc_kernel": 2}
 FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
+
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
+# kernel from one ncu capture on a smaller grid, as bytes per algorithmic FLOP
+# (profiles/bsa_attn_tc_dram_traffic_720p.md).  The full-size figure is scaled
+# by the launch's algorithmic FLOPs, and reported only while the kernel's
+# sources hash to the value they had when the counters were taken.
+ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_fwd.cuh", "tc_common.cuh")
+PROFILED_TRAFFIC = {
+    "bsa_dkdv_tc_kernel": dict(bytes=2814417664 + 1113137152, flops=20362737745920.0, grid="720p-like 24x48x80",
+                               sha256="9a734e2f3077968e16279dbb03b03a1fcb67fa6b172c514a221d09772fc779b5"),
+}
+
+
+def profiled_traffic(kernel, flops_per_launch):
+    rec = PROFILED_TRAFFIC.get(kernel)
+    if rec is None:
+        return None, None
+    import hashlib
+    csrc = os.path.join(ROOT, "dynamic_block_sparse_variance_b200", "csrc")
+    hsh = hashlib.sha256()
+    for f in ATTN_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            hsh.update(fh.read())
+    if hsh.hexdigest() != rec["sha256"]:
+        return None, "kernel changed since the ncu capture"
+    return rec["bytes"] / rec["flops"] * flops_per_launch, (f"ncu capture on the {rec['grid']} grid, scaled by "
+                                                            "algorithmic FLOPs per launch")
 BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel", "bsa_dkdv_tc_kernel", "bsa_dq_tc_kernel")
 
 
@@ -290,8 +317,10 @@ def run_prism(args, rank, world):
         per_launch = KERNEL_FLOP_UNITS[dom_name] * (unit_of[dom_name] if split and dom_name in unit_of else Punit)
         achieved = per_launch / (dom_ms / dom_n * 1e-3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+        traffic, traffic_src = profiled_traffic(dom_name, per_launch)
         roof = dict(kernel=dom_name, bound="tensor", achieved=achieved, peak=peak, unit="TFLOP/s",
-                    frac=achieved / peak, traffic=None, peak_source=f"{peak_src} sustained bf16 (cuBLAS)",
+                    frac=achieved / peak, traffic=traffic, traffic_source=traffic_src,
+                    peak_source=f"{peak_src} sustained bf16 (cuBLAS)",
                     flops_per_launch=per_launch, ms_per_launch=dom_ms / dom_n)
     else:
         roof = dict(kernel=dom_name, bound="hbm", achieved=None, peak=peaks.get("hbm_gbs"), unit="GB/s",
