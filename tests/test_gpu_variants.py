@@ -83,8 +83,8 @@ MODES = {
 }
 
 
-@pytest.mark.parametrize("mode", list(MODES))
-@pytest.mark.parametrize("name", ["aniso8", "mix16"])
+@pytest.mark.parametrize("name,mode", [("aniso8", "fixed444"), ("aniso8", "ratio"), ("aniso8", "fixed444+ratio"),
+                                       ("mix16", "ratio"), ("mix16", "fixed444+ratio")])
 def test_variant_end_to_end(name, mode):
     kw = MODES[mode]
     wl = synth.get_workload(name)
