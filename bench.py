@@ -44,6 +44,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense-attention comparator")
+    ap.add_argument("--no-norms", action="store_true", help="skip the audio-norm producer measurement")
     return ap.parse_args()
 
 
@@ -156,6 +158,76 @@ def profiled_traffic(kernel, flops_per_launch):
     return rec["bytes"] / rec["flops"] * flops_per_launch, (f"ncu capture on the {rec['grid']} grid, scaled by "
                                                             "algorithmic FLOPs per launch")
 BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel", "bsa_dkdv_tc_kernel", "bsa_dq_tc_kernel")
+
+
+def hbm_kernel_bytes(wl, nblk, heads_per_pass_launches):
+    """Algorithmic bytes per step of the HBM-bound kernels (each tensor read or
+    written once; bf16 inputs), for achieved GB/s.  Returns {kernel: bytes}."""
+    t = wl.N * wl.heads * wl.head_dim * 2          # one [N, heads, d] bf16 tensor
+    scores = wl.heads * float(nblk) ** 2 * 4        # one fp32 score matrix per head
+    return {
+        "zone_stats_kernel": t,                      # reads V once
+        "permute_kernel": 4 * 2 * t,                 # Q, K, V, dO: read natural + write permuted
+        "unpermute_kernel": 4 * 2 * t,               # O, dQ, dK, dV
+        "bwd_delta_kernel": 3 * t + wl.N * wl.heads * 4,   # dO, O, O residual in; D out
+        "v_to_f16_kernel": 2 * t,                    # V in, fp16 copy out
+        "block_scores_kernel": scores * heads_per_pass_launches,   # score rows written
+        "row_cut_kernel": scores,                    # score rows read once
+        "emit_kernel": scores,                       # score rows read once
+    }
+
+
+def measure_dense(wl, dev, steps=1):
+    """Dense softmax attention (torch SDPA, bf16) on one head of the same grid,
+    forward + backward, as the comparator for the speedup ratio (measurement
+    only; extrapolated to all heads)."""
+    from torch.nn.attention import SDPBackend, sdpa_kernel
+    import torch.nn.functional as F
+    g = torch.Generator(device=dev).manual_seed(9)
+    q, k, v = (torch.randn(1, 1, wl.N, wl.head_dim, device=dev, dtype=torch.bfloat16, generator=g)
+               .requires_grad_(True) for _ in range(3))
+    do = torch.randn(1, 1, wl.N, wl.head_dim, device=dev, dtype=torch.bfloat16, generator=g)
+    for backend in (SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION):
+        try:
+            with sdpa_kernel([backend]):
+                def once():
+                    o = F.scaled_dot_product_attention(q, k, v)
+                    o.backward(do)
+                once()
+                torch.cuda.synchronize()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for _ in range(steps):
+                    once()
+                e1.record()
+                torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / steps
+            flops = 14.0 * float(wl.N) ** 2 * wl.head_dim
+            return dict(backend=str(backend).split(".")[-1], heads_timed=1, ms_per_head=ms,
+                        ms_all_heads=ms * wl.heads, tflops=flops / (ms * 1e-3) / 1e12)
+        except Exception as exc:  # backend unavailable for this size: try the next
+            err = f"{backend}: {type(exc).__name__}: {str(exc)[:120]}"
+    return dict(unavailable=err)
+
+
+def measure_norms(wl, dev, steps=3):
+    """The audio-norm producer (prism_audio_norms) on [N, heads*d] bf16."""
+    from dynamic_block_sparse_variance_b200 import prism as P
+    C = wl.heads * wl.head_dim
+    g = torch.Generator(device=dev).manual_seed(8)
+    h = torch.randn(wl.N, C, device=dev, dtype=torch.bfloat16, generator=g)
+    a = torch.empty(wl.N, device=dev)
+    P.prism_audio_norms(h, a)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        P.prism_audio_norms(h, a)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del h
+    return dict(ms=ms, bytes=wl.N * C * 2, gbs=wl.N * C * 2 / (ms * 1e-3) / 1e9)
 
 
 # ------------------------------------------------------------ CPU oracle --
@@ -328,6 +400,17 @@ def run_prism(args, rank, world):
     t_fwd = sum(summ.get(k, (0, 0.0))[1] for k in FWD_KERNELS) / args.steps
     t_bwd = sum(summ.get(k, (0, 0.0))[1] for k in BWD_KERNELS) / args.steps
     burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm_peak = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    n_scores = summ.get("block_scores_kernel", (0, 0.0))[0] // max(1, args.steps)
+    n_cut = max(1, summ.get("row_cut_kernel", (0, 0.0))[0] // max(1, args.steps))
+    hbm_bytes = hbm_kernel_bytes(wl, nb, n_scores / n_cut)
+    kernels = {}
+    for k, (n, t) in sorted(summ.items()):
+        rec = dict(launches=n, ms_per_step=t / args.steps)
+        if k in hbm_bytes and t > 0:
+            gbs = hbm_bytes[k] / (t / args.steps * 1e-3) / 1e9
+            rec.update(algorithmic_gb_per_step=hbm_bytes[k] / 1e9, achieved_gbs=gbs, hbm_frac=gbs / hbm_peak)
+        kernels[k] = rec
     value = world * exec_flops / (ms * 1e-3) / 1e12
     out = dict(
         metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
@@ -346,10 +429,19 @@ def run_prism(args, rank, world):
                        flop_density=pairs / (wl.heads * float(wl.N) ** 2),
                        block_density=nnz / (wl.heads * float(nb) ** 2), nblk=nb, nnz=nnz,
                        B_hist={int(b): int((sizes == b).sum().item()) for b in (64, 128, 256)}),
-        kernels={k: dict(launches=n, ms_per_step=t / args.steps) for k, (n, t) in sorted(summ.items())},
+        kernels=kernels,
         gpu_launches=launches,
         clocks=clk,
     )
+    if not args.no_norms and world == 1:
+        nm = measure_norms(wl, dev)
+        nm.update(hbm_frac=nm["gbs"] / hbm_peak, shape=f"[{wl.N}, {wl.heads * wl.head_dim}] bf16")
+        out["audio_norms"] = nm
+    if not args.no_dense and world == 1:
+        dn = measure_dense(wl, dev)
+        if "ms_all_heads" in dn:
+            dn["speedup_vs_dense"] = dn["ms_all_heads"] / ms
+        out["dense_attention"] = dn
     # end-to-end through the public API with host buffers
     if not args.no_e2e:
         out["e2e"] = run_e2e(att, inputs, (O, dq, dk, dv), wl, exec_flops, args, world)

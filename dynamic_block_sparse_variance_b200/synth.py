@@ -77,11 +77,18 @@ TEST_WORKLOADS = {
 }
 
 
+# The 720p grid with a third of the heads: inputs still larger than L2 (0.19 GB
+# per tensor) but a whole layer's buffers within a few GB, the size used for
+# profiler captures that replay each kernel many times.
+PROFILE_WORKLOADS = {
+    "720p-8h": Workload("720p-8h", 24, 48, 80, 8, 128, "bf16", 16, 0.9, 6, 0.06, False, 1.4, 2),
+}
+
+
 def get_workload(name):
-    if name in WORKLOADS:
-        return WORKLOADS[name]
-    if name in TEST_WORKLOADS:
-        return TEST_WORKLOADS[name]
+    for table in (WORKLOADS, TEST_WORKLOADS, PROFILE_WORKLOADS):
+        if name in table:
+            return table[name]
     raise KeyError(name)
 
 
