@@ -324,7 +324,10 @@ def select_row(P_row, top_k, top_p):
     order = sorted(range(n), key=lambda j: (-P_row[j], j))
     n_p = n
     acc = 0.0
-    for pos, j in enumerate(order):
+    # With p >= 1 only the whole row reaches p in exact arithmetic (every
+    # softmax probability is positive); a float64 running sum can round up to
+    # 1 a few blocks early, so that case is taken as the whole row directly.
+    for pos, j in enumerate(order if top_p < 1.0 else ()):
         acc += P_row[j]
         if acc >= top_p:
             n_p = pos + 1

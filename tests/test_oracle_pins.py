@@ -476,3 +476,27 @@ def test_fixed_shape_mode_is_the_uniform_444_tiling():
     # other fixed shapes keep their own volume
     sid, base, blocks = po.assign_blocks(None, None, T, H, W, fixed_shape=13)
     assert (blocks[:, 1] == 256).all() and (np.diff(base) == 2).all()
+
+
+def test_top_p_one_keeps_every_block_even_where_float_sums_reach_one_early():
+    """p = 1: every softmax probability is positive, so no proper prefix has mass 1
+    in exact arithmetic and Top-p is the whole row.  Softmax rows whose float64
+    running sum (in ranking order) reaches 1.0 before the end are common; on such a
+    row the selection must still be the whole row, and p just below 1 stops early."""
+    rng = np.random.default_rng(0)
+    early = None
+    for _ in range(2000):
+        n = int(rng.integers(3, 40))
+        P = po.block_probabilities(rng.normal(0, 1, n) * rng.uniform(0.1, 20))
+        acc = 0.0
+        for pos, j in enumerate(sorted(range(n), key=lambda j: (-P[j], j))):
+            acc += P[j]
+            if acc >= 1.0:
+                if pos + 1 < n:
+                    early = P
+                break
+        if early is not None:
+            break
+    assert early is not None
+    np.testing.assert_array_equal(po.select_row(early, 1, 1.0), np.arange(len(early)))
+    assert len(po.select_row(early, 1, 1.0 - 1e-9)) < len(early)
