@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__res
   // k: absolute, or the ratio form ceil((1 - sparsity) * nblk), at least 1
   const int k_eff = sparsity > 0.f ? max(1, (int)ceil((1.0 - (double)sparsity) * (double)n)) : top_k;
   const unsigned long long kk = (unsigned long long)min(k_eff, n);
-  if (tot < pf) {  // top-p never reached: the whole row
+  // top-p never reached, or p >= 1 (every probability is positive, so only
+  // the whole row has mass 1 exactly): the whole row
+  if (tot < pf || top_p >= 1.f) {
     if (threadIdx.x == 0) {
       cnt[row] = n;
       cut_key[row] = 0xffffffffu;

@@ -213,7 +213,8 @@ int prism_unpermute(const prism_params *p, const uint8_t *shape_id, const void *
  * S_i = Top-k(P_i, k) U Top-p(P_i, p): key blocks ranked by (score
  * descending, index ascending); S_i is the longest of the first min(k, nblk)
  * and the shortest prefix whose mass reaches p (mass summed in 2^-40 fixed
- * point).  k is p->top_k, or comes from p->sparsity and nblk on the device
+ * point; p >= 1 keeps the whole row, the only prefix of mass 1 in exact
+ * arithmetic).  k is p->top_k, or comes from p->sparsity and nblk on the device
  * when that is set.  Output is a CSR per head over rows h*8Z + i, columns
  * ascending.
  *   nblk [1]              in (device), from prism_assign_blocks

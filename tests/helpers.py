@@ -104,3 +104,58 @@ def selection_row_ok(P_row, gpu_sel, ora_sel, top_k, top_p, score_tol=1e-4, mass
             pref = set(order[:len(gs)])
             valid = gs == pref
     return False, valid
+
+
+def check_whole_path(wl, inp, att_kw=None, ora_kw=None, audio=None, zero_grads=()):
+    """Run the whole GPU path (forward + backward) on the CPU inputs `inp` and
+    compare it with the oracle run in the same mode: block layout bit for bit,
+    every selection row exact or a valid near-tie alternative (>= 99% exact),
+    O and dQ, dK, dV within the attention tolerance.  Gradients named in
+    `zero_grads` are exactly zero (the oracle's reference must be zero to
+    rounding); a relative error has no meaning there, so they are held to the
+    max-abs bound alone.  Returns (att, ora, out)."""
+    from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
+    from dynamic_block_sparse_variance_b200 import prism as P
+    from oracle import prism_oracle as po
+    att_kw, ora_kw = dict(att_kw or {}), dict(ora_kw or {})
+    a = inp["audio"] if audio is None else audio
+    a64 = None if a is None else a.numpy().astype(np.float64)
+    ora = po.pipeline(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), wl.T, wl.H, wl.W, a64, wl.top_k, wl.top_p,
+                      **ora_kw)
+    att = PrismSparseAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, **att_kw)
+    cu = lambda t: None if t is None else t.cuda()
+    out = att.forward(cu(inp["q"]), cu(inp["k"]), cu(inp["v"]), cu(a))
+    P.prism_device_status()
+    lay = att.host_layout()
+    np.testing.assert_array_equal(lay["shape_id"], ora["shape_id"])
+    np.testing.assert_array_equal(lay["blocks"], ora["blocks"])
+    nb = len(ora["blocks"])
+    k_eff = po.top_k_from_sparsity(ora_kw["sparsity"], nb) if ora_kw.get("sparsity") else wl.top_k
+    rp_g, cols_g = att.host_csr()
+    scale = ora["scale"]
+    exact = total = 0
+    for h in range(wl.heads):
+        s = po.block_scores(ora["qbar"][h], ora["kbar"][h], scale)
+        for i in range(nb):
+            g = cols_g[h][rp_g[h, i]:rp_g[h, i + 1]]
+            o = ora["cols"][h][ora["row_ptr"][h, i]:ora["row_ptr"][h, i + 1]]
+            ex, ok = selection_row_ok(po.block_probabilities(s[i]), g, o, k_eff, wl.top_p)
+            assert ok, (h, i, g, o)
+            assert len(g) >= min(k_eff, nb)
+            exact += ex
+            total += 1
+    assert exact >= 0.99 * total, f"{exact}/{total} rows bit-exact"
+    bf = lambda t: f64(t.to(torch.bfloat16))
+    pm = {n: po.permute(bf(inp[n]), ora["perm"]) for n in ("q", "k", "v", "dout")}
+    O, _ = po.bsa_forward(pm["q"], pm["k"], pm["v"], ora["blocks"], rp_g, cols_g, scale)
+    assert_close_attn(f64(out), po.unpermute(O, ora["perm"]), "O")
+    dq, dk, dv = att.backward(cu(inp["dout"]))
+    P.prism_device_status()
+    gq, gk, gv = po.bsa_backward(pm["q"], pm["k"], pm["v"], pm["dout"], ora["blocks"], rp_g, cols_g, scale)
+    for got, ref, w in ((dq, gq, "dQ"), (dk, gk, "dK"), (dv, gv, "dV")):
+        if w in zero_grads:
+            assert np.abs(ref).max() < 1e-12, f"{w}: the reference is not zero"
+            assert np.abs(f64(got)).max() <= MAX_ABS_TOL, f"{w}: max-abs {np.abs(f64(got)).max():.3e}"
+        else:
+            assert_close_attn(f64(got), po.unpermute(ref, ora["perm"]), w)
+    return att, ora, out

@@ -105,3 +105,13 @@ def test_audio_norms_host_checks(lib):
     assert lib.prism_audio_norms(None, P.PRISM_BF16, 10, 8, fake, None) == P.PRISM_EINVAL
     assert lib.prism_audio_norms(fake, P.PRISM_BF16, -1, 8, fake, None) == P.PRISM_EINVAL
     assert lib.prism_audio_norms(None, P.PRISM_BF16, 0, 8, None, None) == P.PRISM_OK          # empty: no launch
+
+
+def test_selection_beyond_its_shared_memory_rejected_on_host(lib):
+    """A head's score row is sorted in shared memory: 4 bytes per block, 8 blocks
+    per zone.  8000 zones (T x H x W = 8 x 800 x 640) need 256 KB, beyond the
+    227 KB a CTA can have; the call says so before any launch."""
+    p = P.make_params(8, 800, 640, 1, 64, 4, 0.9)
+    fake = ctypes.c_void_p(0x1000)
+    rc = lib.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, None, 0, fake, fake, 1 << 40, None)
+    assert rc == P.PRISM_EINVAL and b"too many blocks" in lib.prism_last_error()

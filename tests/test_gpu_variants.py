@@ -15,9 +15,8 @@ import torch
 
 from dynamic_block_sparse_variance_b200 import prism as P
 from dynamic_block_sparse_variance_b200 import synth
-from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
 from oracle import prism_oracle as po
-from tests.helpers import assert_close_attn, f64, selection_row_ok
+from tests.helpers import check_whole_path, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -89,42 +88,7 @@ def test_variant_end_to_end(name, mode):
     kw = MODES[mode]
     wl = synth.get_workload(name)
     inp = synth.make_inputs(wl, "cpu", with_dout=True)
-    audio = None if inp["audio"] is None else inp["audio"].numpy().astype(np.float64)
     fixed = kw["fixed_shape"] - 1 if "fixed_shape" in kw else None
-    ora = po.pipeline(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), wl.T, wl.H, wl.W, audio, wl.top_k, wl.top_p,
-                      fixed_shape=fixed, sparsity=kw.get("sparsity"))
-    att = PrismSparseAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, **kw)
-    cu = lambda t: None if t is None else t.cuda()
-    out = att.forward(cu(inp["q"]), cu(inp["k"]), cu(inp["v"]), cu(inp["audio"]))
-    P.prism_device_status()
-    lay = att.host_layout()
-    np.testing.assert_array_equal(lay["shape_id"], ora["shape_id"])
-    np.testing.assert_array_equal(lay["blocks"], ora["blocks"])
+    att, _, _ = check_whole_path(wl, inp, att_kw=kw, ora_kw=dict(fixed_shape=fixed, sparsity=kw.get("sparsity")))
     if fixed is not None:
-        assert (lay["shape_id"] == 3).all()
-    nb = len(ora["blocks"])
-    k_eff = po.top_k_from_sparsity(kw["sparsity"], nb) if "sparsity" in kw else wl.top_k
-    rp_g, cols_g = att.host_csr()
-    # the oracle's probabilities, from its own pooled vectors, for the near-tie check
-    scale = ora["scale"]
-    exact = total = 0
-    for h in range(wl.heads):
-        s = po.block_scores(ora["qbar"][h], ora["kbar"][h], scale)
-        for i in range(nb):
-            g = cols_g[h][rp_g[h, i]:rp_g[h, i + 1]]
-            o = ora["cols"][h][ora["row_ptr"][h, i]:ora["row_ptr"][h, i + 1]]
-            ex, ok = selection_row_ok(po.block_probabilities(s[i]), g, o, k_eff, wl.top_p)
-            assert ok, (h, i, g, o)
-            assert len(g) >= min(k_eff, nb)
-            exact += ex
-            total += 1
-    assert exact >= 0.99 * total, f"{exact}/{total} rows bit-exact"
-    bf = lambda t: f64(t.to(torch.bfloat16))
-    pm = {n: po.permute(bf(inp[n]), ora["perm"]) for n in ("q", "k", "v", "dout")}
-    O, _ = po.bsa_forward(pm["q"], pm["k"], pm["v"], ora["blocks"], rp_g, cols_g, scale)
-    assert_close_attn(f64(out), po.unpermute(O, ora["perm"]), f"O ({mode})")
-    dq, dk, dv = att.backward(cu(inp["dout"]))
-    P.prism_device_status()
-    gq, gk, gv = po.bsa_backward(pm["q"], pm["k"], pm["v"], pm["dout"], ora["blocks"], rp_g, cols_g, scale)
-    for got, ref, w in ((dq, gq, "dQ"), (dk, gk, "dK"), (dv, gv, "dV")):
-        assert_close_attn(f64(got), po.unpermute(ref, ora["perm"]), f"{w} ({mode})")
+        assert (att.host_layout()["shape_id"] == 3).all()
