@@ -38,57 +38,85 @@ struct Load4<float> {
 
 // part[(m * nslab + slab) * 3 + d] = sum over the slab's channels c of
 // (1/8) sum_i (Vbar^{(d)}_{i,c} - mu_c)^2.
+// Each warp streams its time slice row by row with the next row's eight loads
+// issued before the current row is summed (two rows in flight).  Its row sums
+// (the H pool of the slice) go to shared memory as soon as a row is done, so
+// only the T and W sums stay in registers; the cross-warp combines then run in
+// warp order 0..7, the same order of float additions as a sequential sum.
 template <typename Tin>
-__global__ void __launch_bounds__(256) zone_stats_kernel(const Tin *__restrict__ V, int C, int H, int W,
+__global__ void __launch_bounds__(256, 2) zone_stats_kernel(const Tin *__restrict__ V, int C, int H, int W,
                                                          int ZY, int ZX, float *__restrict__ part) {
-  __shared__ float sT[8][kSlab];     // [t][c]: slice sums, one warp per t
-  __shared__ float sH[8][kSlab];     // [y][c]: summed over the eight warps in order
-  __shared__ float sW[8][kSlab];     // [x][c]
+  __shared__ float sT[8][kSlab];      // [t][c]: slice sums, one warp per t
+  __shared__ float sHw[8][8][kSlab];  // [t][y][c]: row sums of each slice
+  __shared__ float sH[8][kSlab];      // [y][c]: summed over the eight warps in order
+  __shared__ float sW[8][kSlab];      // [x][c]
   __shared__ float red[8][3];
   const int slab = blockIdx.x, m = blockIdx.y, nslab = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int zt = m / (ZY * ZX), zy = (m / ZX) % ZY, zx = m % ZX;
   const int c0 = slab * kSlab + lane * 4;
   const bool active = c0 < C;
-  float accT[4] = {0, 0, 0, 0}, accH[8][4], accW[8][4];
+  float accT[4] = {0, 0, 0, 0}, accW[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int c = 0; c < 4; ++c) accH[i][c] = accW[i][c] = 0.f;
+    for (int c = 0; c < 4; ++c) accW[i][c] = 0.f;
   if (active) {
     const int64_t t = zt * kZone + warp;
+    const Tin *base = V + ((t * H + zy * kZone) * W + zx * kZone) * (int64_t)C + c0;
+    const int64_t row_stride = (int64_t)W * C;
+    float v[2][8][4];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) Load4<Tin>::run(base + x * (int64_t)C, v[0][x]);
 #pragma unroll
     for (int y = 0; y < 8; ++y) {
-      const int64_t row = (t * H + zy * kZone + y) * W + zx * kZone;
-      float v[8][4];
+      const int cur = y & 1;
+      if (y + 1 < 8) {
 #pragma unroll
-      for (int x = 0; x < 8; ++x) Load4<Tin>::run(V + (row + x) * C + c0, v[x]);
+        for (int x = 0; x < 8; ++x) Load4<Tin>::run(base + (y + 1) * row_stride + x * (int64_t)C, v[cur ^ 1][x]);
+      }
+      float accH[4] = {0, 0, 0, 0};
 #pragma unroll
       for (int x = 0; x < 8; ++x)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          accT[c] += v[x][c];
-          accH[y][c] += v[x][c];
-          accW[x][c] += v[x][c];
+          accT[c] += v[cur][x][c];
+          accH[c] += v[cur][x][c];
+          accW[x][c] += v[cur][x][c];
         }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sHw[warp][y][lane * 4 + c] = accH[c];
     }
+  } else {
+#pragma unroll
+    for (int y = 0; y < 8; ++y)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) sHw[warp][y][lane * 4 + c] = 0.f;
   }
 #pragma unroll
   for (int c = 0; c < 4; ++c) sT[warp][lane * 4 + c] = accT[c];
-  // fixed-order (warp 0, 1, ..., 7) accumulation of the H and W pools
+  // fixed-order (warp 0, 1, ..., 7) accumulation of the W pools
   for (int w = 0; w < 8; ++w) {
     if (warp == w) {
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const float h0 = w ? sH[i][lane * 4 + c] : 0.f, w0 = w ? sW[i][lane * 4 + c] : 0.f;
-          sH[i][lane * 4 + c] = h0 + accH[i][c];
+          const float w0 = w ? sW[i][lane * 4 + c] : 0.f;
           sW[i][lane * 4 + c] = w0 + accW[i][c];
         }
     }
     __syncthreads();
   }
+  // H pools: row y summed over the warps in order 0..7
+  for (int e = threadIdx.x; e < 8 * kSlab; e += blockDim.x) {
+    const int y = e / kSlab, c = e % kSlab;
+    float h = sHw[0][y][c];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) h += sHw[w][y][c];
+    sH[y][c] = h;
+  }
+  __syncthreads();
   // threads 0..127: channel c of the slab, all three axes
   float var[3] = {0, 0, 0};
   if (threadIdx.x < kSlab && slab * kSlab + (int)threadIdx.x < C) {
