@@ -210,6 +210,27 @@ def measure_dense(wl, dev, steps=1):
     return dict(unavailable=err)
 
 
+def measure_inference(att, inputs, out, fwd_flops, steps=3):
+    """Inference across diffusion steps: a forward that reuses the last step's
+    block layout and selection (permute Q, K, V; attention; unpermute O)."""
+    from dynamic_block_sparse_variance_b200 import prism as P
+    att.forward_reuse(inputs["q"], inputs["k"], inputs["v"], out=out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with P.KernelTrace() as tr:
+        e0.record()
+        for _ in range(steps):
+            att.forward_reuse(inputs["q"], inputs["k"], inputs["v"], out=out)
+        e1.record()
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    summ = tr.summary()
+    attn_ms = sum(summ.get(k, (0, 0.0))[1] for k in FWD_KERNELS) / steps
+    return dict(ms_per_forward=ms, attn_fwd_ms=attn_ms, executed_tflops=fwd_flops / (ms * 1e-3) / 1e12,
+                attn_executed_tflops=fwd_flops / (attn_ms * 1e-3) / 1e12 if attn_ms else None,
+                gpu_launches=sum(n for n, _ in summ.values()) // steps)
+
+
 def measure_norms(wl, dev, steps=3):
     """The audio-norm producer (prism_audio_norms) on [N, heads*d] bf16."""
     from dynamic_block_sparse_variance_b200 import prism as P
@@ -434,6 +455,8 @@ def run_prism(args, rank, world):
         gpu_launches=launches,
         clocks=clk,
     )
+    if world == 1:
+        out["inference"] = measure_inference(att, inputs, O, 4.0 * Punit)
     if not args.no_norms and world == 1:
         nm = measure_norms(wl, dev)
         nm.update(hbm_frac=nm["gbs"] / hbm_peak, shape=f"[{wl.N}, {wl.heads * wl.head_dim}] bf16")

@@ -106,6 +106,20 @@ class PrismSparseAttention:
         P.prism_unpermute(self.p, self.shape_id, self.op, out)
         return out
 
+    def forward_reuse(self, q, k, v, out=None):
+        """Inference across diffusion steps: attention over new Q, K, V with the
+        block layout and the selection of the last forward() (no indicator,
+        assignment, pooling or selection).  Natural-layout output."""
+        P.prism_permute(self.p, self.shape_id, self.zone_blk_base, q, self.qp, None)
+        P.prism_permute(self.p, self.shape_id, self.zone_blk_base, k, self.kp, None)
+        P.prism_permute(self.p, self.shape_id, self.zone_blk_base, v, self.vp, None)
+        P.prism_bsa_fwd(self.p, self.blocks, self.zone_blk_base, self.nblk, self.qp, self.kp, self.vp,
+                        self.row_ptr, self.col, self.op, self.lse, o_res=None, workspace=self.ws_fwd)
+        if out is None:
+            out = torch.empty(self.N, self.heads, self.D, dtype=torch.bfloat16, device=self.device)
+        P.prism_unpermute(self.p, self.shape_id, self.op, out)
+        return out
+
     # -- backward -----------------------------------------------------------
     def _bwd_buffers(self):
         if self._bwd is None:

@@ -92,3 +92,32 @@ def test_variant_end_to_end(name, mode):
     att, _, _ = check_whole_path(wl, inp, att_kw=kw, ora_kw=dict(fixed_shape=fixed, sparsity=kw.get("sparsity")))
     if fixed is not None:
         assert (att.host_layout()["shape_id"] == 3).all()
+
+
+@pytest.mark.parametrize("name", ["aniso8", "mix16"])
+def test_inference_reuses_layout_and_selection(name):
+    """forward_reuse on the inputs of a later step attends over the selection the
+    first step chose: the oracle's attention on the new inputs with the first
+    step's layout and CSR is the reference."""
+    from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
+    from tests.helpers import assert_close_attn
+    wl = synth.get_workload(name)
+    first = synth.make_inputs(wl, "cpu", with_dout=False)
+    g = torch.Generator().manual_seed(77)
+    later = {n: (first[n].float() + 0.3 * torch.randn(first[n].shape, generator=g)).to(first[n].dtype)
+             for n in ("q", "k", "v")}
+    att = PrismSparseAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, training=False)
+    cu = lambda t: None if t is None else t.cuda()
+    att.forward(cu(first["q"]), cu(first["k"]), cu(first["v"]), cu(first["audio"]))
+    lay0, csr0 = att.host_layout(), att.host_csr()
+    out = att.forward_reuse(cu(later["q"]), cu(later["k"]), cu(later["v"]))
+    P.prism_device_status()
+    lay1, csr1 = att.host_layout(), att.host_csr()
+    np.testing.assert_array_equal(lay0["blocks"], lay1["blocks"])
+    for a, b in zip(csr0[1], csr1[1]):
+        np.testing.assert_array_equal(a, b)
+    perm = po.permutation(wl.T, wl.H, wl.W, lay0["shape_id"])
+    pm = {n: po.permute(f64(later[n].to(torch.bfloat16)), perm) for n in ("q", "k", "v")}
+    O, _ = po.bsa_forward(pm["q"], pm["k"], pm["v"], lay0["blocks"].astype(np.int64), csr0[0], csr0[1],
+                          1.0 / np.sqrt(wl.head_dim))
+    assert_close_attn(f64(out), po.unpermute(O, perm), "O with the reused selection")
