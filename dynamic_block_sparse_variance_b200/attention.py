@@ -166,3 +166,112 @@ class PrismSparseAttention:
             out_cols.append(col[r[0]:r[-1]].astype("int64"))
         import numpy as np
         return np.stack(out_rp), out_cols
+
+
+class HostStepper:
+    """Forward + backward steps on inputs that live in pinned host memory.
+
+    The same C-ABI calls as PrismSparseAttention.forward/backward run on the
+    current stream; the host<->device copies run on two copy streams, ordered
+    by CUDA events so that each one overlaps kernels instead of bracketing the
+    step: step i+1's Q, K, V and audio upload as soon as step i has read them
+    (after its permutation), its dO as soon as step i's backward has permuted
+    dO, O downloads while the backward runs, and dQ, dK, dV download while the
+    next step's forward runs.  One device copy of each input and output is
+    enough; nothing waits on the host.
+
+    run(host_inputs, host_outputs): lists (one entry per step) of dicts of
+    pinned host tensors, inputs {q, k, v, audio (or None), dout} and outputs
+    {o, dq, dk, dv}; returns after enqueueing everything (synchronize the
+    current stream, then the copy streams' work is complete too).
+    ``device_buffers`` (optional): the device tensors to stage through, a dict
+    with the same keys (natural layout, the host tensors' shapes and dtypes);
+    by default the stepper allocates its own on the first run.
+    """
+
+    def __init__(self, att: PrismSparseAttention, device_buffers=None):
+        self.att = att
+        self.dev = att.device
+        self.up = torch.cuda.Stream(self.dev)
+        self.down = torch.cuda.Stream(self.dev)
+        self.buf = dict(device_buffers) if device_buffers is not None else None
+
+    def _buffers(self, first):
+        if self.buf is None:
+            shp = (self.att.N, self.att.heads, self.att.D)
+            b = {n: torch.empty(first[n].shape, dtype=first[n].dtype, device=self.dev)
+                 for n in ("q", "k", "v", "dout")}
+            b["audio"] = None if first.get("audio") is None else torch.empty(first["audio"].shape,
+                                                                          dtype=first["audio"].dtype,
+                                                                          device=self.dev)
+            for n in ("o", "dq", "dk", "dv"):
+                b[n] = torch.empty(shp, dtype=torch.bfloat16, device=self.dev)
+            self.buf = b
+        return self.buf
+
+    def _upload(self, host, names, after):
+        with torch.cuda.stream(self.up):
+            if after is not None:
+                self.up.wait_event(after)
+            for n in names:
+                if host.get(n) is not None:
+                    self.buf[n].copy_(host[n], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(self.up)
+        return ev
+
+    def _download(self, names, host, after):
+        with torch.cuda.stream(self.down):
+            self.down.wait_event(after)
+            for n in names:
+                host[n].copy_(self.buf[n], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(self.down)
+        return ev
+
+    def run(self, host_inputs, host_outputs):
+        att = self.att
+        comp = torch.cuda.current_stream(self.dev)
+        b = self._buffers(host_inputs[0])
+        ready_in = self._upload(host_inputs[0], ("q", "k", "v", "audio"), None)
+        ready_do = self._upload(host_inputs[0], ("dout",), None)
+        o_free = grads_free = None
+        for i, (hin, hout) in enumerate(zip(host_inputs, host_outputs)):
+            nxt = host_inputs[i + 1] if i + 1 < len(host_inputs) else None
+            # forward: read the uploaded inputs, then release them for step i+1
+            comp.wait_event(ready_in)
+            if att.fixed_shape == P.PRISM_DYNAMIC_SHAPES:
+                att.indicator(b["v"], b["audio"])
+            att.assign()
+            att.permute(b["q"], b["k"], b["v"])
+            in_free = torch.cuda.Event()
+            in_free.record(comp)
+            if nxt is not None:
+                ready_in = self._upload(nxt, ("q", "k", "v", "audio"), in_free)
+            att.select()
+            att.attend()
+            if o_free is not None:
+                comp.wait_event(o_free)
+            P.prism_unpermute(att.p, att.shape_id, att.op, b["o"])
+            o_ready = torch.cuda.Event()
+            o_ready.record(comp)
+            o_free = self._download(("o",), hout, o_ready)
+            # backward
+            bw = att._bwd_buffers()
+            comp.wait_event(ready_do)
+            P.prism_permute(att.p, att.shape_id, att.zone_blk_base, b["dout"], bw["dop"], None)
+            do_free = torch.cuda.Event()
+            do_free.record(comp)
+            if nxt is not None:
+                ready_do = self._upload(nxt, ("dout",), do_free)
+            att.attend_backward()
+            if grads_free is not None:
+                comp.wait_event(grads_free)
+            for src, n in ((bw["dqp"], "dq"), (bw["dkp"], "dk"), (bw["dvp"], "dv")):
+                P.prism_unpermute(att.p, att.shape_id, src, b[n])
+            g_ready = torch.cuda.Event()
+            g_ready.record(comp)
+            grads_free = self._download(("dq", "dk", "dv"), hout, g_ready)
+        # the caller's stream covers the last downloads
+        comp.wait_event(o_free)
+        comp.wait_event(grads_free)
