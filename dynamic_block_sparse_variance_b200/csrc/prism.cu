@@ -262,6 +262,40 @@ int prism_audio_norms(const void *h, int h_dtype, int64_t N, int C, float *a, pr
   return PRISM_OK;
 }
 
+int prism_zone_records(const prism_params *p, const void *V, int v_dtype, const float *audio, double *records,
+                       void *workspace, size_t ws_bytes, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!V || !records) return fail(PRISM_EINVAL, "zone_records: V and records must be non-NULL");
+  if (!aligned16(V)) return fail(PRISM_EINVAL, "V must be 16-byte aligned");
+  if (v_dtype != PRISM_BF16 && v_dtype != PRISM_F32) return fail(PRISM_EINVAL, "V dtype must be bf16 or f32");
+  IndicatorWs w(d);
+  if (!workspace || ws_bytes < w.total) return fail(PRISM_EINVAL, "indicator workspace too small");
+  cudaStream_t st = as_stream(stream);
+  float *part = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + w.part);
+  dim3 grid(w.nslab, (unsigned)d.Z);
+  if (v_dtype == PRISM_BF16)
+    PRISM_TRACED("zone_stats_kernel", st, zone_stats_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16 *>(V), (int)d.C,
+                                                            d.H, d.W, d.ZY, d.ZX, part));
+  else
+    PRISM_TRACED("zone_stats_kernel", st, zone_stats_kernel<float><<<grid, 256, 0, st>>>(static_cast<const float *>(V), (int)d.C, d.H, d.W, d.ZY,
+                                                    d.ZX, part));
+  PRISM_TRACED("zone_finish_kernel", st, zone_finish_kernel<<<(unsigned)d.Z, 64, 0, st>>>(part, w.nslab, (int)d.C, audio, d.H, d.W, d.ZY, d.ZX, records));
+  return PRISM_OK;
+}
+
+int prism_zone_finalize(const prism_params *p, const double *records, int has_audio, float *g, float *rho,
+                        float *debug, prism_stream stream) {
+  Dims d;
+  int rc = check_params(p, &d);
+  if (rc) return rc;
+  if (!records || !g || !rho) return fail(PRISM_EINVAL, "zone_finalize: records, g and rho must be non-NULL");
+  cudaStream_t st = as_stream(stream);
+  PRISM_TRACED("zone_final_kernel", st, zone_final_kernel<<<1, 1024, 0, st>>>(records, (int)d.Z, has_audio != 0, p->eps, g, rho, debug));
+  return PRISM_OK;
+}
+
 int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, const float *audio, float *g,
                          float *rho, float *debug, void *workspace, size_t ws_bytes, prism_stream stream) {
   Dims d;

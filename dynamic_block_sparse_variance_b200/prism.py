@@ -23,7 +23,7 @@ PRISM_OPT_ATTN_BACKEND, PRISM_OPT_WAIT_LIMIT, PRISM_OPT_DEBUG_STALL = 0, 1, 2
 
 # Entry points declared in include/prism.h, in declaration order.
 ENTRY_POINTS = (
-    "prism_workspace_size", "prism_audio_norms", "prism_zone_indicator", "prism_zone_indicator_noalloc", "prism_assign_blocks",
+    "prism_workspace_size", "prism_audio_norms", "prism_zone_records", "prism_zone_finalize", "prism_zone_indicator", "prism_zone_indicator_noalloc", "prism_assign_blocks",
     "prism_permute",
     "prism_unpermute", "prism_block_select", "prism_bsa_fwd", "prism_bsa_bwd",
     "prism_set_option", "prism_set_trace", "prism_device_status", "prism_last_error",
@@ -78,6 +78,8 @@ def lib():
         sig = {
             "prism_workspace_size": [pp, ctypes.c_int, i64, ctypes.POINTER(sz), ctypes.POINTER(sz)],
             "prism_audio_norms": [_P, ctypes.c_int, i64, ctypes.c_int, _P, _P],
+            "prism_zone_records": [pp, _P, ctypes.c_int, _P, _P, _P, sz, _P],
+            "prism_zone_finalize": [pp, _P, ctypes.c_int, _P, _P, _P, _P],
             "prism_zone_indicator": [pp, _P, ctypes.c_int, _P, _P, _P, _P, _P, sz, _P],
             "prism_zone_indicator_noalloc": [pp, _P, ctypes.c_int, _P, _P, _P, _P, _P],
             "prism_assign_blocks": [pp, _P, _P, _P, _P, _P, _P, _P],
@@ -133,6 +135,21 @@ def prism_audio_norms(h, a):
     """a[n] = ||h[n, :]||_2 for a row-major [N, C] tensor h (bf16 or f32)."""
     _check(lib().prism_audio_norms(_ptr(h), _dtype(h), h.shape[0], h.shape[1] if h.dim() > 1 else 0, _ptr(a),
                                    _stream()))
+
+
+PRISM_ZONE_RECORD = 9
+
+
+def prism_zone_records(p, V, audio, records, workspace):
+    """Per-zone indicator records [Z, 9] float64 of the grid p describes (a T-slab or the whole grid)."""
+    _check(lib().prism_zone_records(ctypes.byref(p), _ptr(V), _dtype(V), _ptr(audio), _ptr(records),
+                                    _ptr(workspace), workspace.numel(), _stream()))
+
+
+def prism_zone_finalize(p, records, has_audio, g, rho, debug=None):
+    """g, rho (and debug) of the whole grid p from the records of all its zones."""
+    _check(lib().prism_zone_finalize(ctypes.byref(p), _ptr(records), int(bool(has_audio)), _ptr(g), _ptr(rho),
+                                     _ptr(debug), _stream()))
 
 
 def prism_zone_indicator(p, V, audio, g, rho, debug, workspace):

@@ -147,6 +147,32 @@ int prism_zone_indicator(const prism_params *p, const void *V, int v_dtype, cons
                          prism_stream stream);
 
 /*
+ * The indicator in two halves, for a grid whose tokens are spread over several
+ * GPUs by T-slabs (slabs of whole 8-frame zone layers; a slab is a grid of its
+ * own and its zones are the full grid's zones m0 .. m0+Z_slab-1, in order):
+ *
+ * prism_zone_records: per zone of the grid described by p (a slab), the
+ *   record of PRISM_ZONE_RECORD doubles
+ *     [sigma2_v,T  sigma2_v,H  sigma2_v,W  info  mean(a)  sigma2_a,T
+ *      sigma2_a,H  sigma2_a,W  max(a)]
+ *   (Method §1: channel-averaged axis variances of the mean-pooled V, their
+ *   sum, and the same pooling of the audio norms; zeros where audio is NULL).
+ *   V, audio, workspace as in prism_zone_indicator; records out [Z, 9].
+ * prism_zone_finalize: from the records of ALL zones of the whole grid
+ *   (p describes the whole grid; the slabs' records concatenated in slab
+ *   order), the grid maxima of info and max(a), then g, rho and debug exactly
+ *   as prism_zone_indicator computes them.  has_audio: nonzero if audio norms
+ *   were given.
+ * prism_zone_records on the whole grid followed by prism_zone_finalize gives
+ * bit for bit the result of prism_zone_indicator.
+ */
+#define PRISM_ZONE_RECORD 9
+int prism_zone_records(const prism_params *p, const void *V, int v_dtype, const float *audio,
+                       double *records, void *workspace, size_t ws_bytes, prism_stream stream);
+int prism_zone_finalize(const prism_params *p, const double *records, int has_audio, float *g, float *rho,
+                        float *debug, prism_stream stream);
+
+/*
  * prism_zone_indicator without any workspace: the same computation, with its
  * scratch (per-zone partial sums) held in a fixed device array inside the
  * library.  It is for callers that cannot allocate device memory at the

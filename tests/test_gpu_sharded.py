@@ -1,0 +1,122 @@
+"""The head-sharded layer on one GPU.
+
+(1) Every rank's stages driven in one process, the exchanges done by slicing:
+the decomposition (slab records -> whole-grid g and rho, slab and whole-grid
+layouts, slab permutation, head groups) must give bit for bit the unsharded
+layer's O, dQ, dK, dV, since every kernel works per zone or per head.
+(2) The layer through TorchDistExchange with a one-rank NCCL group.
+"""
+
+import os
+import socket
+
+import pytest
+import torch
+
+from dynamic_block_sparse_variance_b200 import prism as P
+from dynamic_block_sparse_variance_b200 import synth
+from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
+from dynamic_block_sparse_variance_b200.sharded import ShardedPrismAttention, TorchDistExchange
+
+pytestmark = pytest.mark.gpu
+
+
+def _workload():
+    # 4 zone layers in T, 4 heads: shardable over 2 and 4 ranks, every block volume present
+    return synth.Workload("shard", 32, 16, 24, 4, 128, "bf16", 3, 0.9, 3, 0.15, True, 1.0, 40)
+
+
+def _unsharded(wl, inp):
+    att = PrismSparseAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p)
+    o = att.forward(inp["q"], inp["k"], inp["v"], inp["audio"])
+    dq, dk, dv = att.backward(inp["dout"])
+    P.prism_device_status()
+    return [o, dq, dk, dv]
+
+
+def _emulated(wl, inp, R):
+    sh = [ShardedPrismAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, rank=r, world=R)
+          for r in range(R)]
+    Nl, hpr = sh[0].Nl, sh[0].hpr
+    sl = lambda x, r: None if x is None else x[r * Nl:(r + 1) * Nl]
+    for r, s in enumerate(sh):
+        s.stage_records(sl(inp["v"], r), sl(inp["audio"], r))
+    rec = torch.cat([s.rec_loc for s in sh])
+    for r, s in enumerate(sh):
+        s.rec_all.copy_(rec)
+        s.stage_layout()
+        s.stage_permute(sl(inp["q"], r), sl(inp["k"], r), sl(inp["v"], r))
+
+    def seq_to_heads(get_loc, get_h, rows):
+        for g in range(R):
+            for s in range(R):
+                r0, n = rows(sh[s], s)
+                for hh in range(hpr):
+                    get_h(sh[g])[hh, r0:r0 + n] = get_loc(sh[s])[g * hpr + hh, :n]
+
+    def heads_to_seq(get_h, get_loc, rows):
+        for g in range(R):
+            for s in range(R):
+                r0, n = rows(sh[s], s)
+                for hh in range(hpr):
+                    get_loc(sh[s])[g * hpr + hh, :n] = get_h(sh[g])[hh, r0:r0 + n]
+
+    tok = lambda s, r: (r * Nl, Nl)
+    blk = lambda s, r: s.slab_blocks[r]
+    seq_to_heads(lambda s: s.qp, lambda s: s.inner.qp, tok)
+    seq_to_heads(lambda s: s.kp, lambda s: s.inner.kp, tok)
+    seq_to_heads(lambda s: s.vp, lambda s: s.inner.vp, tok)
+    seq_to_heads(lambda s: s.qbar, lambda s: s.inner.qbar, blk)
+    seq_to_heads(lambda s: s.kbar, lambda s: s.inner.kbar, blk)
+    for s in sh:
+        s.stage_attend()
+    heads_to_seq(lambda s: s.inner.op, lambda s: s.qp, tok)
+    outs = {n: [] for n in ("o", "dq", "dk", "dv")}
+    for r, s in enumerate(sh):
+        o = torch.empty(Nl, wl.heads, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+        s.stage_unpermute(s.qp, o)
+        outs["o"].append(o)
+        s.stage_permute_dout(sl(inp["dout"], r), s.kp)
+    seq_to_heads(lambda s: s.kp, lambda s: s.inner._bwd_buffers()["dop"], tok)
+    for s in sh:
+        s.inner.attend_backward()
+    for n in ("dq", "dk", "dv"):
+        heads_to_seq(lambda s: s.inner._bwd_buffers()[n + "p"], lambda s: s.vp, tok)
+        for s in sh:
+            x = torch.empty(Nl, wl.heads, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+            s.stage_unpermute(s.vp, x)
+            outs[n].append(x)
+    P.prism_device_status()
+    return [torch.cat(outs[n]) for n in ("o", "dq", "dk", "dv")]
+
+
+@pytest.mark.parametrize("R", [2, 4])
+def test_emulated_ranks_equal_the_unsharded_layer(R):
+    wl = _workload()
+    inp = synth.make_inputs(wl, "cuda", with_dout=True)
+    ref = _unsharded(wl, inp)
+    got = _emulated(wl, inp, R)
+    for name, a, b in zip(("O", "dQ", "dK", "dV"), got, ref):
+        assert torch.equal(a, b), name
+
+
+def test_one_rank_nccl_group_equals_the_unsharded_layer():
+    import torch.distributed as dist
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        wl = _workload()
+        inp = synth.make_inputs(wl, "cuda", with_dout=True)
+        ref = _unsharded(wl, inp)
+        layer = ShardedPrismAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, rank=0,
+                                      world=1, exchange=TorchDistExchange(0, 1))
+        o = layer.forward(inp["q"], inp["k"], inp["v"], inp["audio"])
+        dq, dk, dv = layer.backward(inp["dout"])
+        P.prism_device_status()
+        for name, a, b in zip(("O", "dQ", "dK", "dV"), (o, dq, dk, dv), ref):
+            assert torch.equal(a, b), name
+    finally:
+        dist.destroy_process_group()
