@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16 *__r
   s = warp_sum(s);
   if (lane == 0) {
     delta[r] = s;
-    lse2[r] = lse[r] * 1.4426950408889634f;   // LSE in log2 units for the key-side kernel
+    lse2[r] = -(lse[r] * 1.4426950408889634f);   // -LSE in log2 units: the key-side kernel's FMA addend
   }
 }
 

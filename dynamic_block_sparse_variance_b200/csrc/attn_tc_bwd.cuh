@@ -282,9 +282,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < 32; e += 2) {
           const int c = 64 * half + 32 * cc + e;
-          pv[cc][e] = __float_as_uint((c < kv) ? tc::ex2(fmaf(__uint_as_float(pv[cc][e]), sl2, -lse2)) : 0.f);
+          const float2 x = tc::fma2(tc::f2u(pv[cc][e], pv[cc][e + 1]), tc::f2(sl2, sl2), tc::f2(-lse2, -lse2));
+          pv[cc][e] = __float_as_uint((c < kv) ? tc::ex2(x.x) : 0.f);
+          pv[cc][e + 1] = __float_as_uint((c + 1 < kv) ? tc::ex2(x.y) : 0.f);
         }
       }
       // ---- dS = P (dP - D) over dP_n (dQ of the previous tile read dS there before dP_n ran)
@@ -299,9 +301,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
         tc::tmem_ld32(colDP + 32u * cc, dp);   // chunk 0's stores below land on columns already read
         tc::tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[e] = pack_bf16(__uint_as_float(pv[cc][2 * e]) * (__uint_as_float(dp[2 * e]) - dl),
-                            __uint_as_float(pv[cc][2 * e + 1]) * (__uint_as_float(dp[2 * e + 1]) - dl));
+        for (int e = 0; e < 16; ++e) {
+          const float2 d = tc::mul2(tc::f2u(pv[cc][2 * e], pv[cc][2 * e + 1]),
+                                    tc::sub2(tc::f2u(dp[2 * e], dp[2 * e + 1]), tc::f2(dl, dl)));
+          pk[e] = pack_bf16(d.x, d.y);
+        }
         tc::tmem_st16(colDP + 16u * cc, pk);
       }
       tc::tmem_st_wait();
@@ -551,18 +555,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
         uint32_t pk[16];
 #pragma unroll
         for (int g = 0; g < 8; ++g) {   // four query columns at a time
-          float4 L = st_l[8 * cc + g];
+          float4 L = st_l[8 * cc + g];  // -LSE*log2e
           if (!full) {
             const int c0 = 64 * half + 32 * cc + 4 * g;
-            if (c0 + 0 >= qv) L.x = INFINITY;
-            if (c0 + 1 >= qv) L.y = INFINITY;
-            if (c0 + 2 >= qv) L.z = INFINITY;
-            if (c0 + 3 >= qv) L.w = INFINITY;
+            if (c0 + 0 >= qv) L.x = -INFINITY;
+            if (c0 + 1 >= qv) L.y = -INFINITY;
+            if (c0 + 2 >= qv) L.z = -INFINITY;
+            if (c0 + 3 >= qv) L.w = -INFINITY;
           }
-          const float p0 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 0]), sl2, -L.x));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 1]), sl2, -L.y));
-          const float p2 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 2]), sl2, -L.z));
-          const float p3 = tc::ex2(fmaf(__uint_as_float(pv[cc][4 * g + 3]), sl2, -L.w));
+          const float2 x01 = tc::fma2(tc::f2u(pv[cc][4 * g + 0], pv[cc][4 * g + 1]), tc::f2(sl2, sl2), tc::f2(L.x, L.y));
+          const float2 x23 = tc::fma2(tc::f2u(pv[cc][4 * g + 2], pv[cc][4 * g + 3]), tc::f2(sl2, sl2), tc::f2(L.z, L.w));
+          const float p0 = tc::ex2(x01.x);
+          const float p1 = tc::ex2(x01.y);
+          const float p2 = tc::ex2(x23.x);
+          const float p3 = tc::ex2(x23.y);
           pv[cc][4 * g + 0] = __float_as_uint(p0);
           pv[cc][4 * g + 1] = __float_as_uint(p1);
           pv[cc][4 * g + 2] = __float_as_uint(p2);
@@ -589,10 +595,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dkdv_tc_kernel(const __gri
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
           const float4 Dv = st_d[8 * cc + g];   // padding columns have P = 0, so dS = 0 there
-          dk[2 * g] = pack_bf16(__uint_as_float(pv[cc][4 * g + 0]) * (__uint_as_float(dp[4 * g + 0]) - Dv.x),
-                                __uint_as_float(pv[cc][4 * g + 1]) * (__uint_as_float(dp[4 * g + 1]) - Dv.y));
-          dk[2 * g + 1] = pack_bf16(__uint_as_float(pv[cc][4 * g + 2]) * (__uint_as_float(dp[4 * g + 2]) - Dv.z),
-                                    __uint_as_float(pv[cc][4 * g + 3]) * (__uint_as_float(dp[4 * g + 3]) - Dv.w));
+          const float2 d01 = tc::mul2(tc::f2u(pv[cc][4 * g + 0], pv[cc][4 * g + 1]),
+                                      tc::sub2(tc::f2u(dp[4 * g + 0], dp[4 * g + 1]), tc::f2(Dv.x, Dv.y)));
+          const float2 d23 = tc::mul2(tc::f2u(pv[cc][4 * g + 2], pv[cc][4 * g + 3]),
+                                      tc::sub2(tc::f2u(dp[4 * g + 2], dp[4 * g + 3]), tc::f2(Dv.z, Dv.w)));
+          dk[2 * g] = pack_bf16(d01.x, d01.y);
+          dk[2 * g + 1] = pack_bf16(d23.x, d23.y);
         }
         tc::tmem_st16(colDP + 16u * cc, dk);
       }
