@@ -138,8 +138,8 @@ FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
 # sources hash to the value they had when the counters were taken.
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_fwd.cuh", "tc_common.cuh")
 PROFILED_TRAFFIC = {
-    "bsa_dkdv_tc_kernel": dict(bytes=2814417664 + 1113137152, flops=20362737745920.0, grid="720p-like 24x48x80",
-                               sha256="9a734e2f3077968e16279dbb03b03a1fcb67fa6b172c514a221d09772fc779b5"),
+    "bsa_dkdv_tc_kernel": dict(bytes=2814518016 + 1116547072, flops=20362737745920.0, grid="720p-like 24x48x80",
+                               sha256="343f1292417aac6f3a811e33b5053ccd16cd3b0289cd11dacd9429daf45cff04"),
 }
 
 
