@@ -129,9 +129,17 @@ def test_fullsize_sampled_parity(name):
                 sel_of_g.setdefault(int(j), []).append(i)
         assert mismatch <= max(1, nb // 100), f"{mismatch} of {nb} rows differ at near-ties"
         # key blocks whose selectors agree on both sides; few selectors keep the fp64 backward short
+        # (each selecting query block costs a full fp64 attention backward over its whole selection,
+        # seconds at 1080p and 2K): the two with the fewest selectors, and one more drawn at random,
+        # from all of them on the smaller grids and from those with at most 32 selectors on the large ones
         same = sorted((len(v), j) for j, v in sel_of_o.items() if sel_of_g.get(j) == v)
-        keys = [j for _, j in same[:2]] + [j for _, j in same[len(same) // 2: len(same) // 2 + 1]]
-        assert keys
+        assert same
+        keys = [j for _, j in same[:2]]
+        rest = same[2:]
+        if name in ("1080p", "2k"):
+            rest = [c for c in rest if c[0] <= 32] or rest[:1]
+        if rest:
+            keys.append(rest[int(rng.integers(len(rest)))][1])
         qh, kh, vh, doh = (_head(cpu[n], h, perm) for n in ("q", "k", "v", "dout"))
         cols = [np.concatenate(cols_o)]
         for j in keys:
