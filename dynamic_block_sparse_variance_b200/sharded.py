@@ -130,7 +130,12 @@ class ShardedPrismAttention:
         self.Zl = self.Nl // 512
         self.hpr = heads // world
         self.dev = torch.device(device)
-        self.ex = exchange
+        if exchange is None and world > 1:
+            import torch.distributed as dist
+            if not dist.is_initialized():
+                raise RuntimeError("ShardedPrismAttention over several ranks needs torch.distributed initialised "
+                                   "(or an explicit exchange)")
+        self.ex = exchange if exchange is not None else TorchDistExchange(rank, world)
         fixed = kw.get("fixed_shape", P.PRISM_DYNAMIC_SHAPES)
         extra = {k: kw[k] for k in ("tau128", "tau256", "eps", "scale") if k in kw}
         self.p_loc = P.make_params(self.Tl, H, W, heads, head_dim, top_k, top_p, fixed_shape=fixed,
