@@ -130,12 +130,7 @@ class ShardedPrismAttention:
         self.Zl = self.Nl // 512
         self.hpr = heads // world
         self.dev = torch.device(device)
-        if exchange is None and world > 1:
-            import torch.distributed as dist
-            if not dist.is_initialized():
-                raise RuntimeError("ShardedPrismAttention over several ranks needs torch.distributed initialised "
-                                   "(or an explicit exchange)")
-        self.ex = exchange if exchange is not None else TorchDistExchange(rank, world)
+        self._ex = exchange
         fixed = kw.get("fixed_shape", P.PRISM_DYNAMIC_SHAPES)
         extra = {k: kw[k] for k in ("tau128", "tau256", "eps", "scale") if k in kw}
         self.p_loc = P.make_params(self.Tl, H, W, heads, head_dim, top_k, top_p, fixed_shape=fixed,
@@ -202,6 +197,19 @@ class ShardedPrismAttention:
         P.prism_permute(self.p_loc, self.shape_loc, self.zbb_loc, dout_loc, dop_loc, None)
 
     # -- the whole layer through the exchange ----------------------------------
+    @property
+    def ex(self):
+        """The exchange: the one given, else torch.distributed's (which must be initialised
+        when there is more than one rank)."""
+        if self._ex is None:
+            if self.world > 1:
+                import torch.distributed as dist
+                if not dist.is_initialized():
+                    raise RuntimeError("ShardedPrismAttention over several ranks needs torch.distributed "
+                                       "initialised (or an explicit exchange)")
+            self._ex = TorchDistExchange(self.rank, self.world)
+        return self._ex
+
     def forward(self, q_loc, k_loc, v_loc, audio_loc=None, out=None):
         """Natural-layout O of this rank's tokens, all heads: [N/R, heads, d] bf16."""
         ex, inn = self.ex, self.inner
