@@ -139,7 +139,7 @@ FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_fwd.cuh", "tc_common.cuh")
 PROFILED_TRAFFIC = {
     "bsa_dkdv_tc_kernel": dict(bytes=2814518016 + 1116547072, flops=20362737745920.0, grid="720p-like 24x48x80",
-                               sha256="343f1292417aac6f3a811e33b5053ccd16cd3b0289cd11dacd9429daf45cff04"),
+                               sha256="8ba62d61241b0d547e1f6a9a38404fe6617bf5ee92a2eed77516cad647d10788"),
 }
 
 

@@ -281,12 +281,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bsa_dq_tc_kernel(const __grid_
       tc::mbar_arrive(b_sfree);
 #pragma unroll
       for (int cc = 0; cc < 2; ++cc) {
+        if (kv >= 64 * half + 64) {   // no padding key columns in this half (almost every tile)
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int c = 64 * half + 32 * cc + e;
-          const float2 x = tc::fma2(tc::f2u(pv[cc][e], pv[cc][e + 1]), tc::f2(sl2, sl2), tc::f2(-lse2, -lse2));
-          pv[cc][e] = __float_as_uint((c < kv) ? tc::ex2(x.x) : 0.f);
-          pv[cc][e + 1] = __float_as_uint((c + 1 < kv) ? tc::ex2(x.y) : 0.f);
+          for (int e = 0; e < 32; e += 2) {
+            const float2 x = tc::fma2(tc::f2u(pv[cc][e], pv[cc][e + 1]), tc::f2(sl2, sl2), tc::f2(-lse2, -lse2));
+            pv[cc][e] = __float_as_uint(tc::ex2(x.x));
+            pv[cc][e + 1] = __float_as_uint(tc::ex2(x.y));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int c = 64 * half + 32 * cc + e;
+            const float2 x = tc::fma2(tc::f2u(pv[cc][e], pv[cc][e + 1]), tc::f2(sl2, sl2), tc::f2(-lse2, -lse2));
+            pv[cc][e] = __float_as_uint((c < kv) ? tc::ex2(x.x) : 0.f);
+            pv[cc][e + 1] = __float_as_uint((c + 1 < kv) ? tc::ex2(x.y) : 0.f);
+          }
         }
       }
       // ---- dS = P (dP - D) over dP_n (dQ of the previous tile read dS there before dP_n ran)
