@@ -233,8 +233,12 @@ class HostStepper:
         att = self.att
         comp = torch.cuda.current_stream(self.dev)
         b = self._buffers(host_inputs[0])
-        ready_in = self._upload(host_inputs[0], ("q", "k", "v", "audio"), None)
-        ready_do = self._upload(host_inputs[0], ("dout",), None)
+        # the first uploads overwrite the device inputs: after everything already
+        # queued on the caller's stream (an earlier run may still be reading them)
+        start = torch.cuda.Event()
+        start.record(comp)
+        ready_in = self._upload(host_inputs[0], ("q", "k", "v", "audio"), start)
+        ready_do = self._upload(host_inputs[0], ("dout",), start)
         o_free = grads_free = None
         for i, (hin, hout) in enumerate(zip(host_inputs, host_outputs)):
             nxt = host_inputs[i + 1] if i + 1 < len(host_inputs) else None
