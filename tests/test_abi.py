@@ -115,3 +115,36 @@ def test_selection_beyond_its_shared_memory_rejected_on_host(lib):
     fake = ctypes.c_void_p(0x1000)
     rc = lib.prism_block_select(ctypes.byref(p), fake, fake, fake, fake, None, 0, fake, fake, 1 << 40, None)
     assert rc == P.PRISM_EINVAL and b"too many blocks" in lib.prism_last_error()
+
+
+def test_header_is_c99_and_links(lib, tmp_path):
+    """include/prism.h is a C header: a C99 program (-pedantic, warnings as errors)
+    includes it, links the library and calls the host-only entry points."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "prism.h"
+int main(void) {
+  prism_params p = {64, 96, 160, 24, 128, 0.5f, 0.25f, 1e-4f, 32, 0.9f, 0.f, PRISM_FIXED_444, 0.75f};
+  size_t a = 0, b = 0;
+  if (prism_workspace_size(&p, PRISM_WS_SELECT, 0, &a, &b) != PRISM_OK || a == 0 || b < a) return 1;
+  p.T = 7;
+  if (prism_workspace_size(&p, PRISM_WS_SELECT, 0, &a, &b) != PRISM_EINVAL) return 2;
+  if (strstr(prism_last_error(), "multiples of 8") == NULL) return 3;
+  if (prism_audio_norms(NULL, PRISM_BF16, 0, 8, NULL, NULL) != PRISM_OK) return 4;
+  printf("ok\n");
+  return 0;
+}
+''')
+    libdir = os.path.dirname(P.LIB_PATH)
+    exe = tmp_path / "abi"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lprism_b200", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", (out.returncode, out.stdout, out.stderr)
