@@ -51,3 +51,15 @@ def test_no_cluster_multicast():
     beside peer-memory code on multi-GPU nodes)."""
     for path in CSRC.glob("*.cu*"):
         assert ".multicast::cluster" not in path.read_text(), path.name
+
+
+def test_every_launch_is_traced():
+    """Every kernel launch of the library sits inside a PRISM_TRACED statement, so
+    the launch hook (per-kernel CUDA events, the bench's launch count) sees all of
+    them and a rejected launch fails the call at once."""
+    for path in sorted(CSRC.glob("*.cu*")):
+        text = path.read_text()
+        for m in re.finditer(r"<<<", text):
+            stmt_start = max(text.rfind(";", 0, m.start()), text.rfind("{", 0, m.start()),
+                             text.rfind("}", 0, m.start()))
+            assert "PRISM_TRACED(" in text[stmt_start:m.start()], f"{path.name}: untraced launch at {m.start()}"
