@@ -26,7 +26,9 @@ Parity status per function (pins live in tests/test_oracle_pins.py):
   optimal_log2_edges      pinned (sum = S, independent constrained minimisation)
   quantise_shape          pinned (hand-derived cases, product = B, enumeration)
   permutation / pooling   pinned (bijection, box tiling, round trip)
-  block_select            pinned (subset brute force, invariants)
+  block_scores /          pinned (a hand-worked 2x3 case, invariance of each row
+  block_probabilities       under a common shift of the key blocks, torch softmax)
+  block_select            pinned (subset brute force, invariants, the hand case)
   top_k_from_sparsity     pinned (the README's worked ratio: 0.75 keeps 25%)
   assign_blocks (fixed)   pinned (every zone the 4x4x4 box; equals dynamic
                           assignment wherever that picks 4x4x4)

@@ -500,3 +500,71 @@ def test_top_p_one_keeps_every_block_even_where_float_sums_reach_one_early():
     assert early is not None
     np.testing.assert_array_equal(po.select_row(early, 1, 1.0), np.arange(len(early)))
     assert len(po.select_row(early, 1, 1.0 - 1e-9)) < len(early)
+
+
+# ------------------------------------------------------------ block scores --
+
+def test_block_scores_and_probabilities_hand_derived():
+    """Method §3: each pooled query block is scored against every pooled key
+    block of its head, s_ij = scale * Qbar_i . Kbar_j (R10, R11), and P_i is the
+    softmax of row i over the key blocks.  Two query blocks and three key blocks
+    (so a transposed product has the wrong shape), scale 1/2, worked by hand:
+      Qbar_0 = (1, 0): dots with Kbar = (1,1), (2,0), (0,1) are 1, 2, 0
+      Qbar_1 = (0, 2): dots are 2, 0, 2
+    so s_0 = (1/2, 1, 0), s_1 = (1, 0, 1), and
+      P_0 = (e^{1/2}, e, 1) / (1 + e^{1/2} + e),  P_1 = (e, 1, e) / (1 + 2e)."""
+    qbar = np.array([[1.0, 0.0], [0.0, 2.0]])
+    kbar = np.array([[1.0, 1.0], [2.0, 0.0], [0.0, 1.0]])
+    s = po.block_scores(qbar, kbar, 0.5)
+    assert s.shape == (2, 3)
+    np.testing.assert_array_equal(s, [[0.5, 1.0, 0.0], [1.0, 0.0, 1.0]])
+    e = math.e
+    r = math.sqrt(e)
+    P0 = po.block_probabilities(s[0])
+    P1 = po.block_probabilities(s[1])
+    np.testing.assert_allclose(P0, np.array([r, e, 1.0]) / (1.0 + r + e), rtol=1e-15)
+    np.testing.assert_allclose(P1, np.array([e, 1.0, e]) / (1.0 + 2.0 * e), rtol=1e-15)
+    # the softmax runs along the key blocks of one query row: that row sums to 1,
+    # while a column of the first key block does not
+    assert abs(P0.sum() - 1.0) < 1e-15 and abs(P1.sum() - 1.0) < 1e-15
+    assert abs(P0[0] + P1[0] - 1.0) > 0.1
+    # dropping the scale (or doubling it) changes the hand values
+    assert not np.allclose(po.block_probabilities(po.block_scores(qbar, kbar, 1.0)[0]), P0)
+    # the whole-head selection uses the same rows: k = 1, p = 0.5 keeps the most
+    # probable key block of each row (index 1 for row 0; indices 0 and 2 tie for
+    # row 1, and 0 + 2 together pass 0.5, so both are kept)
+    rp, cols, probs = po.block_select(qbar[None], kbar[None], 1, 0.5, 0.5)
+    np.testing.assert_allclose(probs[0], np.stack([P0, P1]), rtol=1e-15)
+    np.testing.assert_array_equal(rp[0], [0, 1, 3])
+    np.testing.assert_array_equal(cols[0], [1, 0, 2])
+
+
+def test_block_probabilities_ignore_a_common_shift_of_the_key_blocks():
+    """Adding one vector u to every pooled key block adds scale * Qbar_i . u to the
+    whole row i, which a softmax over that row's key blocks ignores.  The added
+    amount differs between rows, so a softmax over the wrong axis, or scores built
+    as Kbar Qbar^T, would move.  Rectangular case (5 query blocks, 9 key blocks)."""
+    rng = np.random.default_rng(21)
+    qbar = rng.standard_normal((5, 6))
+    kbar = rng.standard_normal((9, 6))
+    u = 3.0 * rng.standard_normal(6)
+    scale = 0.37
+    s = po.block_scores(qbar, kbar, scale)
+    s_shift = po.block_scores(qbar, kbar + u, scale)
+    assert s.shape == (5, 9)
+    row_shift = s_shift - s
+    np.testing.assert_allclose(row_shift, np.repeat((scale * qbar @ u)[:, None], 9, axis=1), atol=1e-12)
+    assert np.ptp(row_shift[:, 0]) > 1.0      # rows move by different amounts
+    for i in range(5):
+        np.testing.assert_allclose(po.block_probabilities(s_shift[i]), po.block_probabilities(s[i]),
+                                   rtol=1e-12, atol=1e-15)
+
+
+def test_block_probabilities_match_the_library_softmax():
+    """The probability rows against torch's softmax of the same fp64 scores, on rows
+    with large spreads (the max subtraction keeps them finite)."""
+    rng = np.random.default_rng(22)
+    for n in (1, 2, 7, 300):
+        s = rng.standard_normal(n) * 40.0
+        ref = torch.softmax(torch.from_numpy(s), dim=0).numpy()
+        np.testing.assert_allclose(po.block_probabilities(s), ref, rtol=1e-12, atol=1e-300)
