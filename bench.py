@@ -133,7 +133,7 @@ FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
 # kernel from one ncu capture on a smaller grid, as bytes per algorithmic FLOP
-# (profiles/bsa_attn_tc_dram_traffic_720p.md).  The full-size figure is scaled
+# (the counters of a single-kernel capture on the 720p-like grid).  The full-size figure is scaled
 # by the launch's algorithmic FLOPs, and reported only while the kernel's
 # sources hash to the value they had when the counters were taken.
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_fwd.cuh", "tc_common.cuh")

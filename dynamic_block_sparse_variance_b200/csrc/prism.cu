@@ -339,7 +339,8 @@ static std::mutex g_noalloc_mutex;
 static void *g_noalloc_addr[256];   // per device ordinal
 
 // Device address of the fixed scratch on the current device (looked up on the
-// first call for that device).
+// first call for that device and kept until exit; not valid across
+// cudaDeviceReset, which the header states).
 static int noalloc_scratch(void **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

@@ -74,6 +74,8 @@ WORKLOADS = {
 TEST_WORKLOADS = {
     "mix16": Workload("mix16", 16, 32, 32, 3, 128, "bf16", 4, 0.9, 3, 0.15, True, 1.0, 11),
     "aniso8": Workload("aniso8", 8, 24, 40, 2, 64, "bf16", 3, 0.8, 2, 0.2, False, 1.0, 12),
+    # six zones, head_dim 128 (the tensor-core kernels), all three block volumes
+    "smoke128": Workload("smoke128", 8, 16, 24, 2, 128, "bf16", 2, 0.9, 2, 0.2, True, 1.0, 13),
 }
 
 

@@ -187,7 +187,10 @@ int prism_zone_finalize(const prism_params *p, const double *records, int has_au
  *   The fixed array (about 1.8 MiB) is reserved on every GPU that loads the
  *   library until the process exits.  The first call on each device looks up
  *   the array's device address (cudaGetSymbolAddress) with that device
- *   current; make that first call before any stream capture.  All calls share
+ *   current; make that first call before any stream capture.  The address is
+ *   kept until the process exits; cudaDeviceReset would load the library's
+ *   device code again, possibly elsewhere, so this entry point is not
+ *   supported on a device after cudaDeviceReset.  All calls share
  *   the one array: calls that overlap on the GPU (different streams, or
  *   different host threads, without ordering between them) race on it.
  *   Every other argument, layout and error behaves as in prism_zone_indicator.

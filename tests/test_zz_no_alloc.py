@@ -31,8 +31,7 @@ def _run_workspace_version(p, v, audio, Z):
     return g.cpu().numpy(), rho.cpu().numpy(), dbg.cpu().numpy()
 
 
-@pytest.mark.parametrize("name", ["mix16", "720p"])
-def test_noalloc_indicator_matches_workspace_indicator(name):
+def _check_noalloc(name):
     wl = synth.get_workload(name)
     gen = "cpu" if name == "mix16" else "cuda"
     inp = synth.make_inputs(wl, gen, with_dout=False)
@@ -54,6 +53,18 @@ def test_noalloc_indicator_matches_workspace_indicator(name):
         np.testing.assert_allclose(g.cpu().numpy(), g_ref, rtol=2e-4, atol=1e-6)
         np.testing.assert_allclose(rho.cpu().numpy(), rho_ref, rtol=2e-4, atol=1e-6)
         np.testing.assert_allclose(dbg.cpu().numpy(), dbg_ref, rtol=2e-4, atol=1e-8)
+
+
+@pytest.mark.parametrize("name", ["mix16", "720p"])
+def test_noalloc_indicator_matches_workspace_indicator(name):
+    _check_noalloc(name)
+
+
+def test_noalloc_indicator_smaller_grid_after_a_larger_one():
+    """The array keeps what the last call left in it: a small grid run after a
+    large one must read none of the large grid's partial sums."""
+    _check_noalloc("720p")
+    _check_noalloc("mix16")
 
 
 def test_noalloc_indicator_rejects_grids_beyond_its_scratch():
