@@ -11,8 +11,14 @@
 //                      deterministic); a value-binned histogram locates the bin
 //                      where both "count >= min(k, nblk)" and "mass >= p" first
 //                      hold; that bin's members are sorted exactly by (score
-//                      desc, index asc) and walked to the cut.  The cut is
-//                      stored as (key, number of equal keys taken).
+//                      desc, index asc) and walked to the cut.  A crossing
+//                      bin with more members than the sort buffer is binned
+//                      again over its own value range; scores packed so
+//                      tightly that value bins stop separating them (many
+//                      binades close to zero) are then binned by the bits of
+//                      their 32-bit order keys, 10 bits a level, which ends in
+//                      a single key (a run of equal scores, taken by index).
+//                      The cut is stored as (key, number of equal keys taken).
 // scan kernels         row counts -> CSR row_ptr and nnz (int64 checked
 //                      against the column capacity).
 // emit_kernel          one CTA per row: ascending indices of the selected
@@ -26,7 +32,8 @@ namespace prism {
 constexpr int kSelThreads = 512;
 constexpr int kSelBins = 1024;
 constexpr int kSelList = 2048;       // exact-sort buffer for the crossing bin
-constexpr int kSelMaxLevels = 6;     // value-range refinements before giving up
+constexpr int kSelMaxLevels = 6;     // value-range refinements
+constexpr int kSelKeyLevels = 5;     // then order-key refinements, 10 bits a level: 4 reach one key, the 5th takes a run of equal keys
 constexpr double kMassOne = 1099511627776.0;  // 2^40
 
 // Order-preserving map: ascending key <=> descending score.
@@ -180,7 +187,7 @@ __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__res
   // Members of the current level: keys in [klo, khi].
   uint32_t klo = 0u, khi = 0xfffffffeu;
   unsigned long long cnt_before = 0, mass_before = 0;
-  for (int level = 0; level < kSelMaxLevels; ++level) {
+  for (int level = 0; level < kSelMaxLevels + kSelKeyLevels; ++level) {
     // value range of the members
     uint32_t kmin = 0xffffffffu, kmax = 0u;
     for (int j = threadIdx.x; j < n; j += kSelThreads) {
@@ -195,6 +202,16 @@ __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__res
     const float vhi = key_score(kmin), vlo = key_score(kmax);
     const bool all_equal = kmin == kmax;
     const float inv_w = all_equal ? 0.f : (float)kSelBins / (vhi - vlo);
+    // bins: equal slices of the value range, or (after kSelMaxLevels) of the
+    // key range; both are monotone in the key, so a bin's members are a
+    // contiguous key range and bins ascend with descending score
+    const bool by_key = level >= kSelMaxLevels;
+    const int kshift = all_equal ? 0 : max(0, 22 - __clz(kmax - kmin));   // (kmax - kmin) >> kshift < 1024
+    auto bin_of = [&](uint32_t k) -> int {
+      if (all_equal) return 0;
+      if (by_key) return (int)((k - kmin) >> kshift);
+      return min(kSelBins - 1, (int)((vhi - key_score(k)) * inv_w));
+    };
     for (int b = threadIdx.x; b < kSelBins; b += kSelThreads) {
       sh.hc[b] = 0u;
       sh.hm[b] = 0ull;
@@ -204,10 +221,9 @@ __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__res
     for (int j = threadIdx.x; j < n; j += kSelThreads) {
       const uint32_t k = keys[j];
       if (k >= klo && k <= khi) {
-        const float s = key_score(k);
-        const int b = all_equal ? 0 : min(kSelBins - 1, (int)((vhi - s) * inv_w));
+        const int b = bin_of(k);
         atomicAdd(&sh.hc[b], 1u);
-        atomicAdd(&sh.hm[b], block_mass(s, smax, invZ));
+        atomicAdd(&sh.hm[b], block_mass(key_score(k), smax, invZ));
       }
     }
     __syncthreads();
@@ -291,7 +307,7 @@ __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__res
     for (int j = threadIdx.x; j < n; j += kSelThreads) {
       const uint32_t k = keys[j];
       if (k >= klo && k <= khi) {
-        const int b = min(kSelBins - 1, (int)((vhi - key_score(k)) * inv_w));
+        const int b = bin_of(k);
         if (b == fb) {
           bmin = min(bmin, k);
           bmax = max(bmax, k);
@@ -354,7 +370,7 @@ __global__ void __launch_bounds__(kSelThreads) row_cut_kernel(const float *__res
     khi = bmax;
     __syncthreads();
   }
-  if (threadIdx.x == 0) {  // refinement did not converge: latch, keep the whole row
+  if (threadIdx.x == 0) {  // unreachable (the key levels end in one key): latch, keep the whole row
     set_status(PRISM_EBOUNDS);
     cnt[row] = n;
     cut_key[row] = 0xffffffffu;
