@@ -34,6 +34,8 @@ Parity status per function (pins live in tests/test_oracle_pins.py):
                           assignment wherever that picks 4x4x4)
   bsa_forward / backward  pinned (dense attention at k = all via torch SDPA,
                           finite differences, autograd of a dense masked form)
+  bsa_query_block_dq /    pinned (autograd of the dense masked form, on the
+  bsa_key_block_dkdv        rows of the blocks they return)
 """
 
 from __future__ import annotations
@@ -448,6 +450,64 @@ def bsa_backward(q, k, v, dout, blocks, row_ptr, cols, scale, query_blocks=None,
             dq[h, start:start + size] += scale * (dS @ k[h, rows])
             dk[h, rows] += scale * (dS.T @ qi)
     return dq, dk, dv
+
+
+def bsa_query_block_dq(q, k, v, dout, blocks, row_ptr, cols, scale, query_blocks, h=0):
+    """dQ of a few query blocks of head h, the gradient of bsa_forward with respect
+    to those blocks' query rows (for sampled checks on large grids, without
+    whole-grid arrays).  Same algebra as bsa_backward, rows of block i only:
+      P = softmax(scale q_i k_S^T), dP = dO_i v_S^T, D_r = sum_c P_rc dP_rc,
+      dQ_i = scale (P (dP - D)) k_S   over the tokens of S_i.
+    Returns {i: dQ_i [B_i, d] float64}."""
+    out = {}
+    for i in query_blocks:
+        start, size = blocks[i][0], blocks[i][1]
+        sel = cols[h][row_ptr[h, i]:row_ptr[h, i + 1]]
+        rows = _key_rows(blocks, sel)
+        qi = np.asarray(q[h, start:start + size], dtype=np.float64)
+        ks = np.asarray(k[h, rows], dtype=np.float64)
+        logits = scale * (qi @ ks.T)
+        e = np.exp(logits - logits.max(axis=1, keepdims=True))
+        P = e / e.sum(axis=1, keepdims=True)
+        dP = np.asarray(dout[h, start:start + size], dtype=np.float64) @ np.asarray(v[h, rows], dtype=np.float64).T
+        D = (P * dP).sum(axis=1, keepdims=True)
+        out[i] = scale * ((P * (dP - D)) @ ks)
+    return out
+
+
+def bsa_key_block_dkdv(q, k, v, dout, blocks, row_ptr, cols, scale, key_blocks, h=0):
+    """dK and dV of a few key blocks of head h: every query block i whose S_i
+    holds key block j adds
+      dV_j += P[:, j]^T dO_i,   dK_j += scale dS[:, j]^T q_i,
+    with P, dS of query block i formed over all of S_i (the softmax and D_r need
+    the whole row).  Returns {j: (dK_j, dV_j)}, each [B_j, d] float64."""
+    want = {int(j) for j in key_blocks}
+    acc = {j: (np.zeros((blocks[j][1], q.shape[2])), np.zeros((blocks[j][1], q.shape[2]))) for j in want}
+    nb = row_ptr.shape[1] - 1
+    for i in range(nb):
+        sel = [int(j) for j in cols[h][row_ptr[h, i]:row_ptr[h, i + 1]]]
+        hit = [j for j in sel if j in want]
+        if not hit:
+            continue
+        start, size = blocks[i][0], blocks[i][1]
+        rows = _key_rows(blocks, sel)
+        qi = np.asarray(q[h, start:start + size], dtype=np.float64)
+        dOi = np.asarray(dout[h, start:start + size], dtype=np.float64)
+        logits = scale * (qi @ np.asarray(k[h, rows], dtype=np.float64).T)
+        e = np.exp(logits - logits.max(axis=1, keepdims=True))
+        P = e / e.sum(axis=1, keepdims=True)
+        dP = dOi @ np.asarray(v[h, rows], dtype=np.float64).T
+        D = (P * dP).sum(axis=1, keepdims=True)
+        dS = P * (dP - D)
+        col0 = 0
+        for j in sel:
+            bj = blocks[j][1]
+            if j in want:
+                dk, dv = acc[j]
+                dv += P[:, col0:col0 + bj].T @ dOi
+                dk += scale * (dS[:, col0:col0 + bj].T @ qi)
+            col0 += bj
+    return acc
 
 
 def pipeline(Q, K, V, T, H, W, audio, top_k, top_p, scale=None, eps=EPS,

@@ -334,6 +334,32 @@ def test_backward_equals_autograd_of_masked_sdpa():
         np.testing.assert_allclose(dv[h], v.grad.numpy(), rtol=1e-9, atol=1e-12)
 
 
+def test_block_restricted_gradients_equal_autograd_of_masked_sdpa():
+    """dQ of chosen query blocks and dK, dV of chosen key blocks (the forms used
+    for sampled checks on large grids) against torch autograd of SDPA with the
+    block mask, on the rows of those blocks."""
+    pb = _tiny_problem(25)
+    row_ptr, cols = _random_csr(pb["blocks"], pb["heads"], 26, 0.4)
+    scale = 1 / math.sqrt(pb["d"])
+    nb = len(pb["blocks"])
+    for h in range(pb["heads"]):
+        mask = torch.from_numpy(_mask(pb["blocks"], row_ptr, cols, h, pb["N"]))
+        q, k, v = (torch.from_numpy(t[h]).clone().requires_grad_(True) for t in (pb["qp"], pb["kp"], pb["vp"]))
+        out = torch.nn.functional.scaled_dot_product_attention(q[None], k[None], v[None], attn_mask=mask[None])
+        out.backward(torch.from_numpy(pb["dop"][h])[None])
+        picks = [0, nb // 2, nb - 1]
+        dq = po.bsa_query_block_dq(pb["qp"], pb["kp"], pb["vp"], pb["dop"], pb["blocks"], row_ptr, cols, scale,
+                                   picks, h=h)
+        kv = po.bsa_key_block_dkdv(pb["qp"], pb["kp"], pb["vp"], pb["dop"], pb["blocks"], row_ptr, cols, scale,
+                                   picks, h=h)
+        for i in picks:
+            s0, sz = pb["blocks"][i][0], pb["blocks"][i][1]
+            np.testing.assert_allclose(dq[i], q.grad.numpy()[s0:s0 + sz], rtol=1e-9, atol=1e-12)
+            dk_j, dv_j = kv[i]
+            np.testing.assert_allclose(dk_j, k.grad.numpy()[s0:s0 + sz], rtol=1e-9, atol=1e-12)
+            np.testing.assert_allclose(dv_j, v.grad.numpy()[s0:s0 + sz], rtol=1e-9, atol=1e-12)
+
+
 def test_backward_against_finite_differences():
     """Central differences of L = sum(dO * O) on a few entries of q, k, v."""
     pb = _tiny_problem(17, T=8, H=8, W=8, heads=1, d=4)
