@@ -54,6 +54,7 @@ struct TcBwdArgs {
   float scale_log2, scale;
   __nv_bfloat16 *dq, *dk, *dv;
   uint32_t wait_limit;
+  int debug_stall;   // test knob (one-kernel backward): P^T_0 is never signalled, so the MMA wait times out
 };
 
 // Tile of a zone: 128 rows (blocks of 128/256) or 64 rows (blocks of 64).

@@ -223,6 +223,9 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           tc::mma_ts(tO, tPn + 8u * k, tc::desc_adv(dV, 2048u * k), idO, (n > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)   // the low fp16 halves of P, 64 columns further on
+          tc::mma_ts(tO, tPn + 64u + 8u * k, tc::desc_adv(dV, 2048u * k), idO, 1u);
         tc::mma_commit(b_vempty(s));
         tc::mma_commit(b_ofull);
       }
@@ -302,15 +305,17 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        uint32_t pk[16], pl[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
           const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
           pk[e] = pack_f16(p0, p1);
+          pl[e] = pack_f16(p0 - f16_lo(pk[e]), p1 - f16_hi(pk[e]));   // exact residuals, rounded to fp16
         }
         tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
+        tc::tmem_st16(tS(b) + lane_off + 64u + 16u * c, pl);
       }
       l_run += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tmem_st_wait();
@@ -506,6 +511,9 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           tc::mma_ts(tOg, tPg + 8u * k, tc::desc_adv(dV, 2048u * k), idO, (n > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < 8; ++k)   // the low fp16 halves of P, 64 columns further on
+          tc::mma_ts(tOg, tPg + 64u + 8u * k, tc::desc_adv(dV, 2048u * k), idO, 1u);
       };
       auto wait_k = [&](int n) {
         return tc::mbar_wait(b_kfull(n % kTc2Stages), (uint32_t)(n / kTc2Stages) & 1u, abort, limit);
@@ -594,15 +602,17 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        uint32_t pk[16], pl[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
           const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
           r8[e & 7] += p0 + p1;
           pk[e] = pack_f16(p0, p1);
+          pl[e] = pack_f16(p0 - f16_lo(pk[e]), p1 - f16_hi(pk[e]));   // exact residuals, rounded to fp16
         }
         tc::tmem_st16(tS(g) + lane_off + 16u * c, pk);
+        tc::tmem_st16(tS(g) + lane_off + 64u + 16u * c, pl);
       }
       if (n > 0 && __any_sync(0xffffffffu, grow)) {
         // rare: rescale O (S_g(n) was issued after PV_g(n-1), so O has settled;

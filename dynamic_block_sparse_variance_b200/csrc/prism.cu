@@ -11,6 +11,7 @@
 
 #include "attn_mma_bwd.cuh"
 #include "attn_tc_bwd.cuh"
+#include "attn_tc_bwd_fused.cuh"
 #include "indicator.cuh"
 #include "norms.cuh"
 #include "permute.cuh"
@@ -22,6 +23,7 @@ static thread_local std::string t_error;
 static int g_attn_backend = 0;
 static uint32_t g_wait_limit = 0;
 static int g_debug_stall = 0;
+static int g_bwd_kernels = 0;
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
@@ -140,7 +142,7 @@ struct SelectWs {
   }
 };
 struct BwdWs {
-  size_t delta, lse2, ccnt, col_ptr, fill, part, tot, row_idx, total;
+  size_t delta, lse2, ccnt, col_ptr, fill, part, tot, row_idx, dqacc, total;
   int64_t R, nchunk;
   BwdWs(const Dims &d, int64_t col_capacity) {
     R = (int64_t)d.heads * d.cap;
@@ -154,7 +156,9 @@ struct BwdWs {
     part = fill + align256(R * 4);
     tot = part + align256(nchunk * 8);
     row_idx = tot + 256;
-    total = row_idx + align256((size_t)(col_capacity > 0 ? col_capacity : 0) * 4);
+    dqacc = row_idx + align256((size_t)(col_capacity > 0 ? col_capacity : 0) * 4);
+    // head_dim 128: fp32 dQ accumulator of the one-kernel tensor-core backward
+    total = dqacc + (d.D == 128 ? (size_t)d.heads * d.N * 128 * 4 : 0);
   }
 };
 
@@ -190,6 +194,7 @@ int prism_set_option(int option, int64_t value) {
     case PRISM_OPT_ATTN_BACKEND: g_attn_backend = (int)value; return PRISM_OK;
     case PRISM_OPT_WAIT_LIMIT: g_wait_limit = (uint32_t)value; return PRISM_OK;
     case PRISM_OPT_DEBUG_STALL: g_debug_stall = (int)value; return PRISM_OK;
+    case PRISM_OPT_BWD_KERNELS: g_bwd_kernels = (int)value; return PRISM_OK;
     default: return fail(PRISM_EINVAL, "unknown option");
   }
 }
@@ -692,11 +697,22 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
     a.dk = static_cast<__nv_bfloat16 *>(dk);
     a.dv = static_cast<__nv_bfloat16 *>(dv);
     a.wait_limit = g_wait_limit ? g_wait_limit : kDefaultWaitLimit;
-    cudaFuncSetAttribute(bsa_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemBytes);
-    cudaFuncSetAttribute(bsa_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmemBytes);
+    a.debug_stall = g_debug_stall;
     dim3 tgrid((unsigned)(d.Z * 8), d.heads);
-    PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, kBwdThreads, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
-    PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, kBwdThreads, kDqSmemBytes, st>>>(tk, tv, a));
+    if (g_bwd_kernels == 0) {
+      float *dqacc = reinterpret_cast<float *>(ws + w.dqacc);
+      if (cudaMemsetAsync(dqacc, 0, (size_t)d.heads * d.N * 128 * 4, st) != cudaSuccess)
+        return fail(PRISM_ECUDA, "cudaMemsetAsync failed");
+      cudaFuncSetAttribute(bsa_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFbSmemBytes);
+      PRISM_TRACED("bsa_bwd_tc_kernel", st, bsa_bwd_tc_kernel<<<tgrid, kFbThreads, kFbSmemBytes, st>>>(tq, tk, tv, to, a, dqacc));
+      PRISM_TRACED("dq_convert_kernel", st, dq_convert_kernel<<<dim3((unsigned)(d.N / 64), d.heads), 256, 0, st>>>(
+          dqacc, d.N, scale, static_cast<__nv_bfloat16 *>(dq)));
+    } else {
+      cudaFuncSetAttribute(bsa_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemBytes);
+      cudaFuncSetAttribute(bsa_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmemBytes);
+      PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, kBwdThreads, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
+      PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, kBwdThreads, kDqSmemBytes, st>>>(tk, tv, a));
+    }
   } else if (d.D == 128)
     rc = launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
                          row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),

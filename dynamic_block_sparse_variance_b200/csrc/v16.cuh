@@ -69,6 +69,9 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&h);
 }
+// The two fp16 halves of a packed pair, as floats.
+__device__ __forceinline__ float f16_lo(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xffffu))); }
+__device__ __forceinline__ float f16_hi(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u >> 16))); }
 
 // out = fp16(v * 2^e_h), same layout.  Grid (x, heads).
 __global__ void __launch_bounds__(256) v_to_f16_kernel(const uint4 *__restrict__ v, int64_t words_per_head,

@@ -84,6 +84,12 @@ TEST_WORKLOADS = {
 # profiler captures that replay each kernel many times.
 PROFILE_WORKLOADS = {
     "720p-8h": Workload("720p-8h", 24, 48, 80, 8, 128, "bf16", 16, 0.9, 6, 0.06, False, 1.4, 2),
+    # the 1080p grid with 4 heads and the 2K grid with 2 heads: the same
+    # generator and knobs, so each head's selection density and working set
+    # match the full grids' in distribution (heads are independent and the
+    # attention kernels take them one after another), at a few GB per layer
+    "1080p-4h": Workload("1080p-4h", 24, 72, 120, 4, 128, "bf16", 16, 0.95, 8, 0.05, True, 3.9, 3),
+    "2k-2h": Workload("2k-2h", 64, 96, 160, 2, 128, "bf16", 32, 0.9, 12, 0.04, True, 3.7, 4),
 }
 
 

@@ -293,6 +293,14 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
  *   nnz, col_capacity     as returned to / given to prism_block_select
  *   dq, dk, dv            out permuted [heads, N, head_dim] bf16
  *   workspace             >= prism_workspace_size(PRISM_WS_BWD, col_capacity)
+ *                         (head_dim 128 adds an fp32 dQ accumulator of
+ *                         heads * N * 128 * 4 bytes)
+ * head_dim 128 on the tensor cores runs one kernel per key tile that forms dK,
+ * dV and each query tile's part of dQ, summed into the fp32 accumulator by
+ * atomic reductions: dQ may then differ run to run in its last bits (the order
+ * of the fp32 additions is not fixed).  PRISM_OPT_BWD_KERNELS = 1 selects the
+ * two-kernel form instead (a key-side kernel for dK, dV and a query-side one
+ * for dQ that recomputes S and dP), which is bit-reproducible and slower.
  */
 int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
                   const int32_t *nblk, const void *q, const void *k, const void *v, const void *o,
@@ -307,12 +315,17 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
  *   PRISM_OPT_WAIT_LIMIT    polls before a device-side wait gives up and
  *                           latches PRISM_ETIMEOUT; 0 restores the default.
  *   PRISM_OPT_DEBUG_STALL   test hook: when 1 the forward kernel never signals
- *                           its first probability tile, so its bounded wait
+ *                           its first probability tile (nor the one-kernel
+ *                           backward its first P^T tile), so a bounded wait
  *                           must time out (PRISM_ETIMEOUT), with no trap or hang.
+ *   PRISM_OPT_BWD_KERNELS   tensor-core backward: 0 (default) one kernel with
+ *                           dQ summed by fp32 reductions; 1 two kernels, dQ
+ *                           owned by a query-side kernel (bit-reproducible).
  * Returns PRISM_EINVAL for an unknown option. */
 #define PRISM_OPT_ATTN_BACKEND 0
 #define PRISM_OPT_WAIT_LIMIT 1
 #define PRISM_OPT_DEBUG_STALL 2
+#define PRISM_OPT_BWD_KERNELS 3
 int prism_set_option(int option, int64_t value);
 
 /* Kernel-launch trace hook.  When set, the library calls

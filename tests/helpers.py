@@ -1,6 +1,8 @@
 """Shared test utilities: comparisons, CSR conversion, near-tie analysis."""
 
+import contextlib
 import math
+import os
 
 import numpy as np
 import torch
@@ -32,15 +34,36 @@ def rel_rms(a, b):
     return float(np.sqrt(np.mean((a - b) ** 2)) / max(np.sqrt(np.mean(b ** 2)), 1e-30))
 
 
+# Below this magnitude half a bf16 ulp is at most 2^-8, and the max-abs bound
+# is also applied to the raw error.
+RAW_MAX_ABS_BELOW = 2.0
+
+
+def _max_err_below(err, ref, bound):
+    small = np.abs(ref) < bound
+    return float(np.max(err[small])) if small.any() else 0.0
+
+
 def assert_close_attn(got, ref, what):
+    """rel-RMS <= 1e-2; max-abs <= 3e-2 beyond half a bf16 ulp of the exact
+    value, and raw max-abs <= 3e-2 over the entries with |ref| < 2.  With
+    PRISM_PARITY_LOG set, one line per comparison is appended to that file
+    (with the raw max-abs below 2 and below 4)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     rr = rel_rms(got, ref)
     err = np.abs(got - ref)
     ma = float(np.max(err))
     beyond = float(np.max(err - bf16_half_ulp(ref)))
-    assert rr <= REL_RMS_TOL and beyond <= MAX_ABS_TOL, \
-        f"{what}: rel_rms={rr:.3e} max_abs={ma:.3e} beyond half-ulp={beyond:.3e}"
+    raw2 = _max_err_below(err, ref, RAW_MAX_ABS_BELOW)
+    log = os.environ.get("PRISM_PARITY_LOG")
+    if log:
+        with open(log, "a") as fh:
+            fh.write(f"{what}\trel_rms={rr:.3e}\tmax_abs={ma:.3e}\tbeyond_half_ulp={beyond:.3e}\t"
+                     f"max_abs(|ref|<2)={raw2:.3e}\tmax_abs(|ref|<4)={_max_err_below(err, ref, 4.0):.3e}\t"
+                     f"max|ref|={float(np.max(np.abs(ref))):.3e}\n")
+    assert rr <= REL_RMS_TOL and beyond <= MAX_ABS_TOL and raw2 <= MAX_ABS_TOL, \
+        f"{what}: rel_rms={rr:.3e} max_abs={ma:.3e} beyond half-ulp={beyond:.3e} max_abs(|ref|<2)={raw2:.3e}"
     return rr, ma
 
 
@@ -159,3 +182,30 @@ def check_whole_path(wl, inp, att_kw=None, ora_kw=None, audio=None, zero_grads=(
         else:
             assert_close_attn(f64(got), po.unpermute(ref, ora["perm"]), w)
     return att, ora, out
+
+
+@contextlib.contextmanager
+def bwd_kernels(mode):
+    """Run the block with the tensor-core backward in `mode`: 0 the one-kernel
+    form (dQ summed by fp32 reductions), 1 the bit-reproducible two-kernel form."""
+    from dynamic_block_sparse_variance_b200 import prism as P
+    P.prism_set_option(P.PRISM_OPT_BWD_KERNELS, mode)
+    try:
+        yield
+    finally:
+        P.prism_set_option(P.PRISM_OPT_BWD_KERNELS, 0)
+
+
+def assert_dq_consistent(got, ref, what="dQ", rel=1e-3, frac=1e-2):
+    """Two gradient results that may differ in the order of their fp32
+    additions (the one-kernel backward sums dQ partials by atomic reductions)
+    or in roundings of dS: rel-RMS of the difference <= rel and no entry
+    further than frac of the largest |ref| (each result is also held to the
+    oracle tolerance by the parity tests)."""
+    g = got.double().cpu()
+    r = ref.double().cpu()
+    d = (g - r)
+    rr = float(d.norm() / r.norm().clamp_min(1e-30))
+    ma = float(d.abs().max())
+    scale = float(r.abs().max())
+    assert rr <= rel and ma <= frac * scale, f"{what}: rel_rms diff {rr:.3e}, max |diff| {ma:.3e} (max |ref| {scale:.3e})"

@@ -54,10 +54,21 @@ def test_hbm_bytes_count_each_tensor_once():
     assert b["block_scores_kernel"] == 2 * b["row_cut_kernel"]     # scores written twice per step
 
 
+def _sources_hash():
+    import hashlib
+    import os
+    h = hashlib.sha256()
+    for f in bench.ATTN_SOURCES:
+        with open(os.path.join(bench.ROOT, "dynamic_block_sparse_variance_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def test_profiled_traffic_only_for_the_profiled_sources(monkeypatch):
-    rec = bench.PROFILED_TRAFFIC["bsa_dkdv_tc_kernel"]
-    got, src = bench.profiled_traffic("bsa_dkdv_tc_kernel", 2 * rec["flops"])
+    rec = dict(bytes=4.0e9, flops=2.0e13, grid="test grid", sha256=_sources_hash())
+    monkeypatch.setitem(bench.PROFILED_TRAFFIC, "bsa_bwd_tc_kernel", rec)
+    got, src = bench.profiled_traffic("bsa_bwd_tc_kernel", 2 * rec["flops"])
     assert got == 2 * rec["bytes"] and "scaled" in src
     assert bench.profiled_traffic("bsa_dq_tc_kernel", 1.0) == (None, None)
-    monkeypatch.setitem(bench.PROFILED_TRAFFIC, "bsa_dkdv_tc_kernel", dict(rec, sha256="0" * 64))
-    assert bench.profiled_traffic("bsa_dkdv_tc_kernel", 1.0)[0] is None
+    monkeypatch.setitem(bench.PROFILED_TRAFFIC, "bsa_bwd_tc_kernel", dict(rec, sha256="0" * 64))
+    assert bench.profiled_traffic("bsa_bwd_tc_kernel", 1.0)[0] is None

@@ -1,7 +1,9 @@
 """HostStepper (inputs and outputs in pinned host memory, copies overlapped
 with the kernels of neighbouring steps) against the same steps run one by one
-on device tensors.  Every kernel of the path is deterministic, so the outputs
-must agree bit for bit, step by step."""
+on device tensors.  With the two-kernel backward every kernel of the path is
+deterministic, so the outputs must agree bit for bit, step by step; with the
+default one-kernel backward O, dK and dV still must, and dQ (summed by fp32
+reductions in arrival order) to within the spread of that order."""
 
 import pytest
 import torch
@@ -9,12 +11,18 @@ import torch
 from dynamic_block_sparse_variance_b200 import prism as P
 from dynamic_block_sparse_variance_b200 import synth
 from dynamic_block_sparse_variance_b200.attention import HostStepper, PrismSparseAttention
+from tests.helpers import assert_dq_consistent, bwd_kernels
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name,own_buffers", [("mix16", False), ("aniso8", True)])
-def test_host_stepper_matches_step_by_step(name, own_buffers):
+@pytest.mark.parametrize("name,own_buffers,mode", [("mix16", False, 1), ("mix16", False, 0), ("aniso8", True, 1)])
+def test_host_stepper_matches_step_by_step(name, own_buffers, mode):
+    with bwd_kernels(mode):
+        _check_host_stepper(name, own_buffers, exact_dq=mode == 1)
+
+
+def _check_host_stepper(name, own_buffers, exact_dq):
     wl = synth.get_workload(name)
     base = synth.make_inputs(wl, "cpu", with_dout=True)
     g = torch.Generator().manual_seed(5)
@@ -47,4 +55,7 @@ def test_host_stepper_matches_step_by_step(name, own_buffers):
     P.prism_device_status()
     for i in range(len(steps)):
         for n in ("o", "dq", "dk", "dv"):
-            assert torch.equal(outs[i][n], ref[i][n]), (i, n)
+            if n == "dq" and not exact_dq:
+                assert_dq_consistent(outs[i][n], ref[i][n], f"step {i} dQ")
+            else:
+                assert torch.equal(outs[i][n], ref[i][n]), (i, n)

@@ -15,7 +15,8 @@ from dynamic_block_sparse_variance_b200 import prism as P
 from dynamic_block_sparse_variance_b200 import synth
 from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
 from oracle import prism_oracle as po
-from tests.helpers import (assert_close_attn, blocks_to_device, csr_to_device, f64, selection_row_ok)
+from tests.helpers import (assert_close_attn, assert_dq_consistent, blocks_to_device, bwd_kernels, csr_to_device,
+                           f64, selection_row_ok)
 
 pytestmark = pytest.mark.gpu
 CASES = ["tiny", "aniso8", "mix16"]
@@ -175,15 +176,18 @@ def test_bsa_forward(name):
     np.testing.assert_allclose(f64(att.lse), L, rtol=0, atol=2e-2)
 
 
-@pytest.mark.parametrize("name", CASES)
-def test_bsa_backward(name):
+@pytest.mark.parametrize("name,mode", [(c, 0) for c in CASES] + [("mix16", 1)])
+def test_bsa_backward(name, mode):
+    """mode 0: the default backward (one tensor-core kernel for head_dim 128,
+    dQ by fp32 reductions); mode 1: the two-kernel tensor-core backward."""
     wl, inp, ora = problem(name)
     att = make_att(wl)
     pm = _oracle_layout_on_gpu(att, ora, inp, wl)
     att.attend()
     b = att._bwd_buffers()
     b["dop"].copy_(torch.from_numpy(pm["dout"]).to(torch.bfloat16))
-    att.attend_backward()
+    with bwd_kernels(mode):
+        att.attend_backward()
     P.prism_device_status()
     dq, dk, dv = po.bsa_backward(pm["q"], pm["k"], pm["v"], pm["dout"], ora["blocks"], ora["row_ptr"],
                                  ora["cols"], ora["scale"])
@@ -296,3 +300,31 @@ def test_forward_v_scale_is_exact():
     assert torch.equal(att.op[1].float(), torch.zeros_like(o_ref[1]))
     assert torch.equal(att.op_res[1].float(), torch.zeros_like(r_ref[1]))
     assert torch.equal(att.op[0].float(), o_ref[0]) and torch.equal(att.op[2].float(), o_ref[2])
+
+
+def test_one_kernel_backward_matches_the_two_kernel_backward():
+    """On the same layout, selection and forward, the one-kernel backward's dV
+    equals the two-kernel form's bit for bit (same products, same elementwise
+    arithmetic, same order).  dK and dQ differ by the two-kernel form's
+    coarser dS (one bf16 rounding, where the one-kernel form keeps dS as a
+    bf16 pair of about 16 bits) and, for dQ, by the order of the fp32 sums;
+    the one-kernel dK is the same bit for bit on every run."""
+    wl, inp, ora = problem("mix16")
+    att = make_att(wl)
+    pm = _oracle_layout_on_gpu(att, ora, inp, wl)
+    att.attend()
+    b = att._bwd_buffers()
+    b["dop"].copy_(torch.from_numpy(pm["dout"]).to(torch.bfloat16))
+    outs = {}
+    for mode in (1, 0, 0):
+        with bwd_kernels(mode):
+            att.attend_backward()
+        P.prism_device_status()
+        outs.setdefault(mode, []).append({n: b[n].clone() for n in ("dqp", "dkp", "dvp")})
+    two, one = outs[1][0], outs[0]
+    for run in one:
+        assert torch.equal(run["dvp"], two["dvp"])
+        assert_dq_consistent(run["dkp"], two["dkp"], "dK", rel=5e-3, frac=2e-2)
+        assert_dq_consistent(run["dqp"], two["dqp"], "dQ", rel=5e-3, frac=2e-2)
+    assert torch.equal(one[0]["dkp"], one[1]["dkp"])
+    assert_dq_consistent(one[0]["dqp"], one[1]["dqp"])   # two runs of the one-kernel form

@@ -5,11 +5,16 @@ the decomposition (slab records -> whole-grid g and rho, slab and whole-grid
 layouts, slab permutation, head groups) must give bit for bit the unsharded
 layer's O, dQ, dK, dV, since every kernel works per zone or per head.
 (2) The layer through TorchDistExchange with a one-rank NCCL group.
+(3) The emulated two-rank layer against the fp64 oracle on the same seeded
+inputs: the whole grid's g and rho on every rank, the block layout exactly,
+every selection row exact or a valid near-tie alternative, and O, dQ, dK, dV
+within rel-RMS 1e-2 and max-abs 3e-2 (beyond half a bf16 ulp).
 """
 
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 
@@ -17,6 +22,8 @@ from dynamic_block_sparse_variance_b200 import prism as P
 from dynamic_block_sparse_variance_b200 import synth
 from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
 from dynamic_block_sparse_variance_b200.sharded import ShardedPrismAttention, TorchDistExchange
+from oracle import prism_oracle as po
+from tests.helpers import assert_close_attn, bwd_kernels, f64, selection_row_ok
 
 pytestmark = pytest.mark.gpu
 
@@ -34,7 +41,7 @@ def _unsharded(wl, inp):
     return [o, dq, dk, dv]
 
 
-def _emulated(wl, inp, R):
+def _emulated(wl, inp, R, ranks=None):
     sh = [ShardedPrismAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, rank=r, world=R)
           for r in range(R)]
     Nl, hpr = sh[0].Nl, sh[0].hpr
@@ -87,6 +94,8 @@ def _emulated(wl, inp, R):
             s.stage_unpermute(s.vp, x)
             outs[n].append(x)
     P.prism_device_status()
+    if ranks is not None:
+        ranks.extend(sh)
     return [torch.cat(outs[n]) for n in ("o", "dq", "dk", "dv")]
 
 
@@ -94,8 +103,9 @@ def _emulated(wl, inp, R):
 def test_emulated_ranks_equal_the_unsharded_layer(R):
     wl = _workload()
     inp = synth.make_inputs(wl, "cuda", with_dout=True)
-    ref = _unsharded(wl, inp)
-    got = _emulated(wl, inp, R)
+    with bwd_kernels(1):   # bit-reproducible dQ
+        ref = _unsharded(wl, inp)
+        got = _emulated(wl, inp, R)
     for name, a, b in zip(("O", "dQ", "dK", "dV"), got, ref):
         assert torch.equal(a, b), name
 
@@ -110,13 +120,55 @@ def test_one_rank_nccl_group_equals_the_unsharded_layer():
     try:
         wl = _workload()
         inp = synth.make_inputs(wl, "cuda", with_dout=True)
-        ref = _unsharded(wl, inp)
-        layer = ShardedPrismAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, rank=0,
-                                      world=1, exchange=TorchDistExchange(0, 1))
-        o = layer.forward(inp["q"], inp["k"], inp["v"], inp["audio"])
-        dq, dk, dv = layer.backward(inp["dout"])
+        with bwd_kernels(1):   # bit-reproducible dQ
+            ref = _unsharded(wl, inp)
+            layer = ShardedPrismAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, rank=0,
+                                          world=1, exchange=TorchDistExchange(0, 1))
+            o = layer.forward(inp["q"], inp["k"], inp["v"], inp["audio"])
+            dq, dk, dv = layer.backward(inp["dout"])
         P.prism_device_status()
         for name, a, b in zip(("O", "dQ", "dK", "dV"), (o, dq, dk, dv), ref):
             assert torch.equal(a, b), name
     finally:
         dist.destroy_process_group()
+
+
+def test_emulated_ranks_against_the_oracle():
+    wl = _workload()
+    inp = synth.make_inputs(wl, "cpu", with_dout=True)
+    cu = {n: (None if t is None else t.cuda()) for n, t in inp.items()}
+    sh = []
+    o, dq, dk, dv = _emulated(wl, cu, 2, ranks=sh)
+    a64 = inp["audio"].numpy().astype(np.float64)
+    ora = po.pipeline(f64(inp["q"]), f64(inp["k"]), f64(inp["v"]), wl.T, wl.H, wl.W, a64, wl.top_k, wl.top_p)
+    for s in sh:   # every rank finalised the whole grid from the gathered slab records
+        np.testing.assert_allclose(f64(s.inner.g), ora["ind"]["g"], rtol=2e-4, atol=1e-6)
+        np.testing.assert_allclose(f64(s.inner.rho), ora["ind"]["rho"], rtol=2e-4, atol=1e-6)
+        lay = s.inner.host_layout()
+        np.testing.assert_array_equal(lay["shape_id"], ora["shape_id"])
+        np.testing.assert_array_equal(lay["blocks"], ora["blocks"])
+    # the head groups' selections, as one per-head CSR
+    nb = len(ora["blocks"])
+    rp_g, cols_g = [], []
+    for s in sh:
+        rp, cols = s.inner.host_csr()
+        rp_g += list(rp)
+        cols_g += cols
+    rp_g = np.stack(rp_g)
+    exact = 0
+    for h in range(wl.heads):
+        S = po.block_scores(ora["qbar"][h], ora["kbar"][h], ora["scale"])
+        for i in range(nb):
+            g = cols_g[h][rp_g[h, i]:rp_g[h, i + 1]]
+            r = ora["cols"][h][ora["row_ptr"][h, i]:ora["row_ptr"][h, i + 1]]
+            ex, ok = selection_row_ok(po.block_probabilities(S[i]), g, r, wl.top_k, wl.top_p)
+            assert ok, (h, i, g, r)
+            exact += ex
+    assert exact >= 0.99 * wl.heads * nb
+    # attention on the selection the ranks made
+    pm = {n: po.permute(f64(inp[n].to(torch.bfloat16)), ora["perm"]) for n in ("q", "k", "v", "dout")}
+    O, _ = po.bsa_forward(pm["q"], pm["k"], pm["v"], ora["blocks"], rp_g, cols_g, ora["scale"])
+    assert_close_attn(f64(o), po.unpermute(O, ora["perm"]), "sharded O")
+    gq, gk, gv = po.bsa_backward(pm["q"], pm["k"], pm["v"], pm["dout"], ora["blocks"], rp_g, cols_g, ora["scale"])
+    for got, ref, w in ((dq, gq, "dQ"), (dk, gk, "dK"), (dv, gv, "dV")):
+        assert_close_attn(f64(got), po.unpermute(ref, ora["perm"]), "sharded " + w)

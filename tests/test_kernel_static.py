@@ -12,7 +12,7 @@ import re
 import pytest
 
 CSRC = pathlib.Path(__file__).resolve().parents[1] / "dynamic_block_sparse_variance_b200" / "csrc"
-SOURCES = ["attn_tc_fwd.cuh", "attn_tc_bwd.cuh"]
+SOURCES = ["attn_tc_fwd.cuh", "attn_tc_bwd.cuh", "attn_tc_bwd_fused.cuh"]
 
 
 def _kernels(text):
@@ -43,7 +43,7 @@ def test_every_declared_barrier_is_initialised_once(src):
             assert inits.count(b) == 1, f"{src}:{name}: barrier {b} initialised {inits.count(b)} times"
         for b in set(inits):
             assert b in declared, f"{src}:{name}: initialises undeclared barrier {b}"
-    assert seen >= 2
+    assert seen >= 1
 
 
 def test_no_cluster_multicast():
