@@ -125,12 +125,11 @@ def executed_pairs(att):
 
 # Algorithmic tensor-core FLOPs of each attention kernel, in units of
 # P = sum_h sum_i sum_{j in S_i} B_i B_j d: forward 4P (QK^T, PV); the
-# one-kernel backward 10P (S, dP, dV, dK, dQ); in the two-kernel backward the
+# tensor-core backward 10P (S, dP, dV, dK, dQ); in the warp-MMA backward the
 # key-side kernel 8P (S, dP, dV, dK) and the query-side one 2P (dQ; its S and
 # dP recomputation is extra work and not counted).
 KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_fwd_tc_kernel": 4, "bsa_fwd_tc2_kernel": 4,
-                     "bsa_dkdv_mma_kernel": 8,
-                     "bsa_dkdv_tc_kernel": 8, "bsa_dq_mma_kernel": 2, "bsa_dq_tc_kernel": 2, "bsa_bwd_tc_kernel": 10}
+                     "bsa_dkdv_mma_kernel": 8, "bsa_dq_mma_kernel": 2, "bsa_bwd_tc_kernel": 10}
 FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
@@ -138,8 +137,7 @@ FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
 # (the counters of a single-kernel capture on the 720p-like grid).  The full-size figure is scaled
 # by the launch's algorithmic FLOPs, and reported only while the kernel's
 # sources hash to the value they had when the counters were taken.
-ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_bwd_fused.cuh", "attn_tc_fwd.cuh",
-                "tc_common.cuh")
+ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_fwd.cuh", "tc_common.cuh", "v16.cuh")
 PROFILED_TRAFFIC = {}
 
 
@@ -157,8 +155,7 @@ def profiled_traffic(kernel, flops_per_launch):
         return None, "kernel changed since the ncu capture"
     return rec["bytes"] / rec["flops"] * flops_per_launch, (f"ncu capture on the {rec['grid']} grid, scaled by "
                                                             "algorithmic FLOPs per launch")
-BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel", "bsa_dkdv_tc_kernel", "bsa_dq_tc_kernel",
-               "bsa_bwd_tc_kernel", "dq_convert_kernel")
+BWD_KERNELS = ("bsa_dkdv_mma_kernel", "bsa_dq_mma_kernel", "bsa_bwd_tc_kernel", "dq_convert_kernel")
 
 
 def hbm_kernel_bytes(wl, nblk, heads_per_pass_launches):
@@ -171,7 +168,10 @@ def hbm_kernel_bytes(wl, nblk, heads_per_pass_launches):
         "permute_kernel": 4 * 2 * t,                 # Q, K, V, dO: read natural + write permuted
         "unpermute_kernel": 4 * 2 * t,               # O, dQ, dK, dV
         "bwd_delta_kernel": 3 * t + wl.N * wl.heads * 4,   # dO, O, O residual in; D out
+        "bwd_stats_tc_kernel": 3 * t + wl.N * wl.heads * 16,   # dO, O, O residual, LSE in; D, m, inv out
         "v_to_f16_kernel": 2 * t,                    # V in, fp16 copy out
+        "head_absmax2_kernel": 2 * t,                # V, dO read once
+        "to_f16x2_kernel": 4 * t,                    # V, dO in, fp16 copies out
         "dq_convert_kernel": 3 * t,                  # fp32 dQ accumulator in, bf16 dQ out
         "block_scores_kernel": scores * heads_per_pass_launches,   # score rows written
         "row_cut_kernel": scores,                    # score rows read once

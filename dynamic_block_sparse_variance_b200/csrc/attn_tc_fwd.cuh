@@ -7,11 +7,18 @@
 //               S_n = Q K_n^T (A, B from shared memory) into one of two S
 //               buffers, and O += P_n V_n with P_n read from tensor memory.
 //   warps 2..5  softmax, one thread per query row (its TMEM lane): S row ->
-//               running max (log2 domain, rescaled lazily only when the max
-//               grows by more than 2^8) -> P = exp2(.) as fp16 written back over
-//               S -> row sum; final normalisation, O (bf16 + residual) and LSE.
+//               running max (log2 domain, an integer, moved lazily only when
+//               the max grows by more than 2^8) -> P = exp2(.) truncated to
+//               11 significant bits, written back over S as fp16 -> row sum
+//               of those values; final normalisation, O (bf16 + residual), LSE.
 // The PV product is fp16 x fp16: V comes as fp16 scaled per head by 2^e_h
 // (see v16.cuh) and the epilogue folds 2^-e_h into 1/l.
+// Why the integer max and the sum of truncated P: O is then exactly
+// sum_c t(2^(x_c - m)) v_c / l for any integer m (truncation to 11 bits
+// commutes with scaling by a power of two), so the backward, given only the
+// LSE, truncates its own exp2(x_c - m') to the same values and its P matches
+// the P that formed O.  The row sums D = rowsum(dO o O) of the backward are then
+// consistent with its dS = P (dP - D), whose rows must sum to zero.
 // MMA order S_0, S_1, PV_0, S_2, PV_1, ... lets QK^T of step n+1 run while the
 // softmax of step n is computed.  Every wait is bounded; a stalled wait raises
 // a CTA-wide abort, latches PRISM_ETIMEOUT and the CTA drains and frees TMEM.
@@ -223,9 +230,6 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           tc::mma_ts(tO, tPn + 8u * k, tc::desc_adv(dV, 2048u * k), idO, (n > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)   // the low fp16 halves of P, 64 columns further on
-          tc::mma_ts(tO, tPn + 64u + 8u * k, tc::desc_adv(dV, 2048u * k), idO, 1u);
         tc::mma_commit(b_vempty(s));
         tc::mma_commit(b_ofull);
       }
@@ -275,12 +279,15 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
         for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
       float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= sl2;
-      // lazy rescaling: only rows whose max grew by more than 2^8 move m_run
+      // lazy rescaling: only rows whose max grew by more than 2^8 move m_run,
+      // which stays an integer, so every rescale is an exact power of two
       const bool grow = mx > m_run + 8.f;
-      const float alpha = grow ? tc::ex2(m_run - mx) : 1.f;
+      float alpha = 1.f;
       if (grow) {
+        const float m_new = ceilf(mx);
+        alpha = pow2_or_zero(m_run - m_new);
         l_run *= alpha;
-        m_run = mx;
+        m_run = m_new;
       }
       if (n > 0 && __any_sync(0xffffffffu, grow)) {
         // O is rescaled once every earlier P V has landed (rows that did not
@@ -305,17 +312,17 @@ __global__ void __launch_bounds__(192, 1) bsa_fwd_tc_kernel(const __grid_constan
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16], pl[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
-          r8[e & 7] += p0 + p1;
+          // P truncated to 11 significant bits: exactly the fp16 operand of the
+          // product, and l sums the same values
+          const float p0 = trunc11(tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run)));
+          const float p1 = trunc11(tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run)));
           pk[e] = pack_f16(p0, p1);
-          pl[e] = pack_f16(p0 - f16_lo(pk[e]), p1 - f16_hi(pk[e]));   // exact residuals, rounded to fp16
+          r8[e & 7] += p0 + p1;
         }
         tc::tmem_st16(tS(b) + lane_off + 16u * c, pk);
-        tc::tmem_st16(tS(b) + lane_off + 64u + 16u * c, pl);
       }
       l_run += ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       tc::tmem_st_wait();
@@ -511,9 +518,6 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
 #pragma unroll
         for (int k = 0; k < 8; ++k)
           tc::mma_ts(tOg, tPg + 8u * k, tc::desc_adv(dV, 2048u * k), idO, (n > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)   // the low fp16 halves of P, 64 columns further on
-          tc::mma_ts(tOg, tPg + 64u + 8u * k, tc::desc_adv(dV, 2048u * k), idO, 1u);
       };
       auto wait_k = [&](int n) {
         return tc::mbar_wait(b_kfull(n % kTc2Stages), (uint32_t)(n / kTc2Stages) & 1u, abort, limit);
@@ -591,28 +595,30 @@ __global__ void __launch_bounds__(kTc2Threads, 1) bsa_fwd_tc2_kernel(const __gri
         for (int e = 0; e < 32; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(raw[c][e]));
       float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx *= sl2;
-      const bool grow = mx > m_run + 8.f;
-      const float alpha = grow ? tc::ex2(m_run - mx) : 1.f;
+      const bool grow = mx > m_run + 8.f;   // integer m_run, exact power-of-two rescales
+      float alpha = 1.f;
       if (grow) {
+        const float m_new = ceilf(mx);
+        alpha = pow2_or_zero(m_run - m_new);
         l_run *= alpha;
-        m_run = mx;
+        m_run = m_new;
       }
       float r8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16], pl[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run));
-          const float p1 = tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run));
-          r8[e & 7] += p0 + p1;
+          // P truncated to 11 significant bits: exactly the fp16 operand of the
+          // product, and l sums the same values
+          const float p0 = trunc11(tc::ex2(fmaf(__uint_as_float(raw[c][2 * e]), sl2, -m_run)));
+          const float p1 = trunc11(tc::ex2(fmaf(__uint_as_float(raw[c][2 * e + 1]), sl2, -m_run)));
           pk[e] = pack_f16(p0, p1);
-          pl[e] = pack_f16(p0 - f16_lo(pk[e]), p1 - f16_hi(pk[e]));   // exact residuals, rounded to fp16
+          r8[e & 7] += p0 + p1;
         }
         tc::tmem_st16(tS(g) + lane_off + 16u * c, pk);
-        tc::tmem_st16(tS(g) + lane_off + 64u + 16u * c, pl);
       }
       if (n > 0 && __any_sync(0xffffffffu, grow)) {
         // rare: rescale O (S_g(n) was issued after PV_g(n-1), so O has settled;

@@ -11,7 +11,6 @@
 
 #include "attn_mma_bwd.cuh"
 #include "attn_tc_bwd.cuh"
-#include "attn_tc_bwd_fused.cuh"
 #include "indicator.cuh"
 #include "norms.cuh"
 #include "permute.cuh"
@@ -23,7 +22,6 @@ static thread_local std::string t_error;
 static int g_attn_backend = 0;
 static uint32_t g_wait_limit = 0;
 static int g_debug_stall = 0;
-static int g_bwd_kernels = 0;
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda).
@@ -142,23 +140,28 @@ struct SelectWs {
   }
 };
 struct BwdWs {
-  size_t delta, lse2, ccnt, col_ptr, fill, part, tot, row_idx, dqacc, total;
+  size_t delta, lse2, stat_inv, ccnt, col_ptr, fill, part, tot, row_idx, amax, f16, dqacc, total;
   int64_t R, nchunk;
   BwdWs(const Dims &d, int64_t col_capacity) {
     R = (int64_t)d.heads * d.cap;
     nchunk = (R + kScanChunk - 1) / kScanChunk;
-    // D and LSE*log2e, each padded by 128 entries for whole-tile bulk copies
+    const size_t rows = (size_t)d.heads * d.N;
+    // D, -LSE*log2e (warp-MMA path) or the integer shift m (tensor-core path),
+    // and 2^(m - LSE*log2e): each padded by 128 entries for whole-tile bulk copies
     delta = 0;
-    lse2 = align256(((size_t)d.heads * d.N + 128) * 4);
-    ccnt = lse2 + align256(((size_t)d.heads * d.N + 128) * 4);
+    lse2 = align256((rows + 128) * 4);
+    stat_inv = lse2 + align256((rows + 128) * 4);
+    ccnt = stat_inv + align256((rows + 128) * 4);
     col_ptr = ccnt + align256(R * 4);
     fill = col_ptr + align256((R + 1) * 4);
     part = fill + align256(R * 4);
     tot = part + align256(nchunk * 8);
     row_idx = tot + 256;
-    dqacc = row_idx + align256((size_t)(col_capacity > 0 ? col_capacity : 0) * 4);
-    // head_dim 128: fp32 dQ accumulator of the one-kernel tensor-core backward
-    total = dqacc + (d.D == 128 ? (size_t)d.heads * d.N * 128 * 4 : 0);
+    amax = row_idx + align256((size_t)(col_capacity > 0 ? col_capacity : 0) * 4);
+    f16 = amax + align256((size_t)d.heads * 2 * 4);
+    // head_dim 128 (tensor cores): fp16 copies of V and dO and the fp32 dQ accumulator
+    dqacc = f16 + (d.D == 128 ? 2 * rows * 128 * 2 : 0);
+    total = dqacc + (d.D == 128 ? rows * 128 * 4 : 0);
   }
 };
 
@@ -194,7 +197,6 @@ int prism_set_option(int option, int64_t value) {
     case PRISM_OPT_ATTN_BACKEND: g_attn_backend = (int)value; return PRISM_OK;
     case PRISM_OPT_WAIT_LIMIT: g_wait_limit = (uint32_t)value; return PRISM_OK;
     case PRISM_OPT_DEBUG_STALL: g_debug_stall = (int)value; return PRISM_OK;
-    case PRISM_OPT_BWD_KERNELS: g_bwd_kernels = (int)value; return PRISM_OK;
     default: return fail(PRISM_EINVAL, "unknown option");
   }
 }
@@ -648,10 +650,33 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
   auto Ores = static_cast<const __nv_bfloat16 *>(o_res);
   if (o_res && !aligned16(o_res)) return fail(PRISM_EINVAL, "bwd: o_res must be 16-byte aligned");
   const int64_t rows = (int64_t)d.heads * d.N;
-  if (d.D == 128)
+  const bool tc_path = d.D == 128 && g_attn_backend == 0;
+  float *stat_inv = reinterpret_cast<float *>(ws + w.stat_inv);
+  uint32_t *amax = reinterpret_cast<uint32_t *>(ws + w.amax);
+  uint8_t *f16 = ws + w.f16;
+  const size_t tensor_bytes = (size_t)rows * 128 * 2;
+  if (tc_path) {
+    // per-head maxima of V and dO and their scaled fp16 copies, then D and the P factors
+    Tensors2 t2;
+    const void *srcs[2] = {v, dout};
+    for (int z = 0; z < 2; ++z) {
+      t2.src[z] = static_cast<const uint4 *>(srcs[z]);
+      t2.dst[z] = reinterpret_cast<uint4 *>(f16 + z * tensor_bytes);
+    }
+    const int64_t words = d.N * 16;   // 16-byte words per head
+    const unsigned gx = (unsigned)std::max<int64_t>(1, std::min<int64_t>((words + 1023) / 1024, (148 * 8 + d.heads - 1) / d.heads));
+    if (cudaMemsetAsync(amax, 0, (size_t)d.heads * 2 * 4, st) != cudaSuccess)
+      return fail(PRISM_ECUDA, "cudaMemsetAsync failed");
+    PRISM_TRACED("head_absmax2_kernel", st, head_absmax2_kernel<<<dim3(gx, d.heads, 2), 256, 0, st>>>(t2, words, d.heads, amax));
+    PRISM_TRACED("to_f16x2_kernel", st, to_f16x2_kernel<<<dim3(gx, d.heads, 2), 256, 0, st>>>(t2, words, d.heads, amax));
+    PRISM_TRACED("bwd_stats_tc_kernel", st, bwd_stats_tc_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+        O, Ores, dO, lse, rows, delta, lse2, stat_inv));
+    cudaMemsetAsync(stat_inv + rows, 0, 128 * 4, st);
+  } else if (d.D == 128) {
     PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<128><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, lse, rows, delta, lse2));
-  else
+  } else {
     PRISM_TRACED("bwd_delta_kernel", st, bwd_delta_kernel<64><<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(O, Ores, dO, lse, rows, delta, lse2));
+  }
   cudaMemsetAsync(delta + rows, 0, 128 * 4, st);
   cudaMemsetAsync(lse2 + rows, 0, 128 * 4, st);
   cudaMemsetAsync(ccnt, 0, w.R * 4, st);
@@ -670,49 +695,39 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
   auto Q = static_cast<const __nv_bfloat16 *>(q), K = static_cast<const __nv_bfloat16 *>(k),
        Vv = static_cast<const __nv_bfloat16 *>(v);
   const float scale = eff_scale(p);
-  if (d.D == 128 && g_attn_backend == 0) {
+  if (tc_path) {
     CUtensorMap tq, tk, tv, to;
-    const uint64_t rows = (uint64_t)d.heads * d.N;
-    if (!make_tile_map(&tq, q, rows) || !make_tile_map(&tk, k, rows) || !make_tile_map(&tv, v, rows) ||
-        !make_tile_map(&to, dout, rows))
+    const uint64_t nrows = (uint64_t)rows;
+    if (!make_tile_map(&tq, q, nrows) || !make_tile_map(&tk, k, nrows) ||
+        !make_tile_map(&tv, f16, nrows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) ||
+        !make_tile_map(&to, f16 + tensor_bytes, nrows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16))
       return fail(PRISM_ECUDA, "cuTensorMapEncodeTiled failed");
     TcBwdArgs a;
     a.blocks = blocks;
     a.zone_blk_base = zone_blk_base;
-    a.row_ptr = row_ptr;
-    a.col = col;
     a.col_ptr = col_ptr;
     a.row_idx = row_idx;
-    a.lse = lse;
-    a.delta = delta;
-    a.lse2_pad = lse2;
+    a.stat_m = lse2;
+    a.stat_inv = stat_inv;
     a.delta_pad = delta;
+    a.amax = amax;
+    a.heads = d.heads;
     a.N = d.N;
     a.cap = d.cap;
     a.scale = scale;
     a.scale_log2 = scale * kLog2e;
-    a.q = Q;
-    a.dout = dO;
-    a.dq = static_cast<__nv_bfloat16 *>(dq);
     a.dk = static_cast<__nv_bfloat16 *>(dk);
     a.dv = static_cast<__nv_bfloat16 *>(dv);
     a.wait_limit = g_wait_limit ? g_wait_limit : kDefaultWaitLimit;
     a.debug_stall = g_debug_stall;
     dim3 tgrid((unsigned)(d.Z * 8), d.heads);
-    if (g_bwd_kernels == 0) {
-      float *dqacc = reinterpret_cast<float *>(ws + w.dqacc);
-      if (cudaMemsetAsync(dqacc, 0, (size_t)d.heads * d.N * 128 * 4, st) != cudaSuccess)
-        return fail(PRISM_ECUDA, "cudaMemsetAsync failed");
-      cudaFuncSetAttribute(bsa_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFbSmemBytes);
-      PRISM_TRACED("bsa_bwd_tc_kernel", st, bsa_bwd_tc_kernel<<<tgrid, kFbThreads, kFbSmemBytes, st>>>(tq, tk, tv, to, a, dqacc));
-      PRISM_TRACED("dq_convert_kernel", st, dq_convert_kernel<<<dim3((unsigned)(d.N / 64), d.heads), 256, 0, st>>>(
-          dqacc, d.N, scale, static_cast<__nv_bfloat16 *>(dq)));
-    } else {
-      cudaFuncSetAttribute(bsa_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmemBytes);
-      cudaFuncSetAttribute(bsa_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSmemBytes);
-      PRISM_TRACED("bsa_dkdv_tc_kernel", st, bsa_dkdv_tc_kernel<<<tgrid, kBwdThreads, kKvSmemBytes, st>>>(tq, tk, tv, to, a));
-      PRISM_TRACED("bsa_dq_tc_kernel", st, bsa_dq_tc_kernel<<<tgrid, kBwdThreads, kDqSmemBytes, st>>>(tk, tv, a));
-    }
+    float *dqacc = reinterpret_cast<float *>(ws + w.dqacc);
+    if (cudaMemsetAsync(dqacc, 0, (size_t)rows * 128 * 4, st) != cudaSuccess)
+      return fail(PRISM_ECUDA, "cudaMemsetAsync failed");
+    cudaFuncSetAttribute(bsa_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kFbSmemBytes);
+    PRISM_TRACED("bsa_bwd_tc_kernel", st, bsa_bwd_tc_kernel<<<tgrid, kFbThreads, kFbSmemBytes, st>>>(tq, tk, tv, to, a, dqacc));
+    PRISM_TRACED("dq_convert_kernel", st, dq_convert_kernel<<<dim3((unsigned)(d.N / 64), d.heads), 256, 0, st>>>(
+        dqacc, d.N, scale, static_cast<__nv_bfloat16 *>(dq)));
   } else if (d.D == 128)
     rc = launch_bwd_attn<128>(d, grid, st, Q, K, Vv, dO, lse, delta, blocks, zone_blk_base, row_ptr, col, col_ptr,
                          row_idx, scale, static_cast<__nv_bfloat16 *>(dq), static_cast<__nv_bfloat16 *>(dk),

@@ -29,6 +29,10 @@ __host__ __device__ __forceinline__ int v16_exponent(uint32_t maxbits) {
 __device__ __forceinline__ float pow2f(int e) {
   return __uint_as_float((uint32_t)(e + 127) << 23);
 }
+// 2^d exactly for an integer-valued d <= 0 (d = -inf or d < -126 give 0).
+__device__ __forceinline__ float pow2_or_zero(float d) {
+  return d >= -126.f ? pow2f((int)d) : 0.f;
+}
 
 // Per-head max |v| of a permuted [heads, N*128] bf16 tensor, as the bf16 bit
 // pattern (abs values of finite bf16 order like their bits).  vmax must be
@@ -72,6 +76,10 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 // The two fp16 halves of a packed pair, as floats.
 __device__ __forceinline__ float f16_lo(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u & 0xffffu))); }
 __device__ __forceinline__ float f16_hi(uint32_t u) { return __half2float(__ushort_as_half((unsigned short)(u >> 16))); }
+
+// x with its 13 low significand bits cleared (rounded toward zero to 11
+// significant bits): exactly an fp16 value when in fp16's normal range.
+__device__ __forceinline__ float trunc11(float x) { return __uint_as_float(__float_as_uint(x) & 0xffffe000u); }
 
 // out = fp16(v * 2^e_h), same layout.  Grid (x, heads).
 __global__ void __launch_bounds__(256) v_to_f16_kernel(const uint4 *__restrict__ v, int64_t words_per_head,

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libprism_b200.so")
 PRISM_OK, PRISM_EINVAL, PRISM_ECAPACITY, PRISM_ECUDA, PRISM_ETIMEOUT, PRISM_EBOUNDS = 0, -1, -2, -3, -4, -5
 PRISM_BF16, PRISM_F32 = 0, 1
 PRISM_WS_INDICATOR, PRISM_WS_SELECT, PRISM_WS_FWD, PRISM_WS_BWD = 0, 1, 2, 3
-PRISM_OPT_ATTN_BACKEND, PRISM_OPT_WAIT_LIMIT, PRISM_OPT_DEBUG_STALL, PRISM_OPT_BWD_KERNELS = 0, 1, 2, 3
+PRISM_OPT_ATTN_BACKEND, PRISM_OPT_WAIT_LIMIT, PRISM_OPT_DEBUG_STALL = 0, 1, 2
 
 # Entry points declared in include/prism.h, in declaration order.
 ENTRY_POINTS = (

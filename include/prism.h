@@ -293,14 +293,17 @@ int prism_bsa_fwd(const prism_params *p, const prism_block *blocks, const int32_
  *   nnz, col_capacity     as returned to / given to prism_block_select
  *   dq, dk, dv            out permuted [heads, N, head_dim] bf16
  *   workspace             >= prism_workspace_size(PRISM_WS_BWD, col_capacity)
- *                         (head_dim 128 adds an fp32 dQ accumulator of
- *                         heads * N * 128 * 4 bytes)
+ *                         (head_dim 128 adds fp16 copies of V and dO and an
+ *                         fp32 dQ accumulator: heads * N * 128 * 8 bytes)
  * head_dim 128 on the tensor cores runs one kernel per key tile that forms dK,
  * dV and each query tile's part of dQ, summed into the fp32 accumulator by
  * atomic reductions: dQ may then differ run to run in its last bits (the order
- * of the fp32 additions is not fixed).  PRISM_OPT_BWD_KERNELS = 1 selects the
- * two-kernel form instead (a key-side kernel for dK, dV and a query-side one
- * for dQ that recomputes S and dP), which is bit-reproducible and slower.
+ * of the fp32 additions is not fixed); dK and dV are reproducible.  Its
+ * dP and dV products take fp16 copies of V and dO scaled per head by powers
+ * of two (exact for bf16 inputs; entries of magnitude 2^75 or more are outside
+ * that range), the others bf16.  It needs O
+ * and lse from the tensor-core forward, whose truncated fp16 probabilities it
+ * reproduces (the rows of dS then sum to zero as they do in exact arithmetic).
  */
 int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_t *zone_blk_base,
                   const int32_t *nblk, const void *q, const void *k, const void *v, const void *o,
@@ -315,17 +318,13 @@ int prism_bsa_bwd(const prism_params *p, const prism_block *blocks, const int32_
  *   PRISM_OPT_WAIT_LIMIT    polls before a device-side wait gives up and
  *                           latches PRISM_ETIMEOUT; 0 restores the default.
  *   PRISM_OPT_DEBUG_STALL   test hook: when 1 the forward kernel never signals
- *                           its first probability tile (nor the one-kernel
+ *                           its first probability tile (nor the tensor-core
  *                           backward its first P^T tile), so a bounded wait
  *                           must time out (PRISM_ETIMEOUT), with no trap or hang.
- *   PRISM_OPT_BWD_KERNELS   tensor-core backward: 0 (default) one kernel with
- *                           dQ summed by fp32 reductions; 1 two kernels, dQ
- *                           owned by a query-side kernel (bit-reproducible).
  * Returns PRISM_EINVAL for an unknown option. */
 #define PRISM_OPT_ATTN_BACKEND 0
 #define PRISM_OPT_WAIT_LIMIT 1
 #define PRISM_OPT_DEBUG_STALL 2
-#define PRISM_OPT_BWD_KERNELS 3
 int prism_set_option(int option, int64_t value);
 
 /* Kernel-launch trace hook.  When set, the library calls

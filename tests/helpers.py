@@ -1,6 +1,5 @@
 """Shared test utilities: comparisons, CSR conversion, near-tie analysis."""
 
-import contextlib
 import math
 import os
 
@@ -184,24 +183,12 @@ def check_whole_path(wl, inp, att_kw=None, ora_kw=None, audio=None, zero_grads=(
     return att, ora, out
 
 
-@contextlib.contextmanager
-def bwd_kernels(mode):
-    """Run the block with the tensor-core backward in `mode`: 0 the one-kernel
-    form (dQ summed by fp32 reductions), 1 the bit-reproducible two-kernel form."""
-    from dynamic_block_sparse_variance_b200 import prism as P
-    P.prism_set_option(P.PRISM_OPT_BWD_KERNELS, mode)
-    try:
-        yield
-    finally:
-        P.prism_set_option(P.PRISM_OPT_BWD_KERNELS, 0)
-
-
 def assert_dq_consistent(got, ref, what="dQ", rel=1e-3, frac=1e-2):
-    """Two gradient results that may differ in the order of their fp32
-    additions (the one-kernel backward sums dQ partials by atomic reductions)
-    or in roundings of dS: rel-RMS of the difference <= rel and no entry
-    further than frac of the largest |ref| (each result is also held to the
-    oracle tolerance by the parity tests)."""
+    """Two dQ results that may differ in the order of their fp32 additions
+    (the tensor-core backward sums dQ partials by atomic reductions): rel-RMS
+    of the difference <= rel and no entry further than frac of the largest
+    |ref| (each result is also held to the oracle tolerance by the parity
+    tests)."""
     g = got.double().cpu()
     r = ref.double().cpu()
     d = (g - r)

@@ -69,6 +69,6 @@ def test_profiled_traffic_only_for_the_profiled_sources(monkeypatch):
     monkeypatch.setitem(bench.PROFILED_TRAFFIC, "bsa_bwd_tc_kernel", rec)
     got, src = bench.profiled_traffic("bsa_bwd_tc_kernel", 2 * rec["flops"])
     assert got == 2 * rec["bytes"] and "scaled" in src
-    assert bench.profiled_traffic("bsa_dq_tc_kernel", 1.0) == (None, None)
+    assert bench.profiled_traffic("bsa_dq_mma_kernel", 1.0) == (None, None)
     monkeypatch.setitem(bench.PROFILED_TRAFFIC, "bsa_bwd_tc_kernel", dict(rec, sha256="0" * 64))
     assert bench.profiled_traffic("bsa_bwd_tc_kernel", 1.0)[0] is None

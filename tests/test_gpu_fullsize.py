@@ -8,12 +8,12 @@ for the exact selectors of sampled key blocks), and the outputs those samples
 determine: O and LSE and dQ of sampled query blocks, dK and dV of sampled key
 blocks.  Query blocks are drawn from a few heads, stratified by block volume
 (at 1080p and 2K: 256 (head, block) pairs); key blocks are the two with the
-fewest selectors and those at the median and 90th percentile of the selector
-count (and its maximum below 2K), each checked against every query block that
+fewest selectors and the one at the median selector count (below 2K also the
+90th percentile and the maximum), each checked against every query block that
 selects it.
 Discrete results are compared exactly (selections up to near-ties); attention
 outputs within rel-RMS 1e-2, max-abs 3e-2 beyond half a bf16 ulp and raw
-max-abs 3e-2 where |ref| < 4.
+max-abs 3e-2 where |ref| < 2.
 """
 
 import math
@@ -165,13 +165,13 @@ def test_fullsize_sampled_parity(name):
         assert mismatch <= max(1, nb // 100), f"{mismatch} of {nb} rows differ at near-ties"
         t0 = _phase(name, "oracle selection of one head", t0)
         # key blocks whose selectors agree on both sides, by selector count: the two
-        # with the fewest, and those at the median and the 90th percentile (and the
-        # top below 2K, where its hundreds of selectors each cost a whole fp64 row)
+        # with the fewest and the median; below 2K also the 90th percentile and the
+        # top (at 2K those hold 500 to 1000 selectors, each a whole fp64 row here)
         same = sorted((len(v), j) for j, v in sel_of_o.items() if sel_of_g.get(j) == v)
         assert len(same) >= 5
-        idx = {0, 1, len(same) // 2, int(0.9 * (len(same) - 1))}
+        idx = {0, 1, len(same) // 2}
         if name != "2k":
-            idx.add(len(same) - 1)
+            idx |= {int(0.9 * (len(same) - 1)), len(same) - 1}
         keys = [same[t][1] for t in sorted(idx)]
         qh, kh, vh, doh = (_head(cpu[n], h, perm) for n in ("q", "k", "v", "dout"))
         kv = po.bsa_key_block_dkdv(qh, kh, vh, doh, blocks, rp_o, [np.concatenate(cols_o)], scale, keys)

@@ -3,7 +3,8 @@
 (1) Every rank's stages driven in one process, the exchanges done by slicing:
 the decomposition (slab records -> whole-grid g and rho, slab and whole-grid
 layouts, slab permutation, head groups) must give bit for bit the unsharded
-layer's O, dQ, dK, dV, since every kernel works per zone or per head.
+layer's O, dK, dV, since every kernel works per zone or per head, and its dQ
+to within the spread of the fp32 reduction order that sums dQ.
 (2) The layer through TorchDistExchange with a one-rank NCCL group.
 (3) The emulated two-rank layer against the fp64 oracle on the same seeded
 inputs: the whole grid's g and rho on every rank, the block layout exactly,
@@ -23,7 +24,7 @@ from dynamic_block_sparse_variance_b200 import synth
 from dynamic_block_sparse_variance_b200.attention import PrismSparseAttention
 from dynamic_block_sparse_variance_b200.sharded import ShardedPrismAttention, TorchDistExchange
 from oracle import prism_oracle as po
-from tests.helpers import assert_close_attn, bwd_kernels, f64, selection_row_ok
+from tests.helpers import assert_close_attn, assert_dq_consistent, f64, selection_row_ok
 
 pytestmark = pytest.mark.gpu
 
@@ -103,11 +104,13 @@ def _emulated(wl, inp, R, ranks=None):
 def test_emulated_ranks_equal_the_unsharded_layer(R):
     wl = _workload()
     inp = synth.make_inputs(wl, "cuda", with_dout=True)
-    with bwd_kernels(1):   # bit-reproducible dQ
-        ref = _unsharded(wl, inp)
-        got = _emulated(wl, inp, R)
+    ref = _unsharded(wl, inp)
+    got = _emulated(wl, inp, R)
     for name, a, b in zip(("O", "dQ", "dK", "dV"), got, ref):
-        assert torch.equal(a, b), name
+        if name == "dQ":
+            assert_dq_consistent(a, b)
+        else:
+            assert torch.equal(a, b), name
 
 
 def test_one_rank_nccl_group_equals_the_unsharded_layer():
@@ -120,15 +123,17 @@ def test_one_rank_nccl_group_equals_the_unsharded_layer():
     try:
         wl = _workload()
         inp = synth.make_inputs(wl, "cuda", with_dout=True)
-        with bwd_kernels(1):   # bit-reproducible dQ
-            ref = _unsharded(wl, inp)
-            layer = ShardedPrismAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, rank=0,
-                                          world=1, exchange=TorchDistExchange(0, 1))
-            o = layer.forward(inp["q"], inp["k"], inp["v"], inp["audio"])
-            dq, dk, dv = layer.backward(inp["dout"])
+        ref = _unsharded(wl, inp)
+        layer = ShardedPrismAttention(wl.T, wl.H, wl.W, wl.heads, wl.head_dim, wl.top_k, wl.top_p, rank=0,
+                                      world=1, exchange=TorchDistExchange(0, 1))
+        o = layer.forward(inp["q"], inp["k"], inp["v"], inp["audio"])
+        dq, dk, dv = layer.backward(inp["dout"])
         P.prism_device_status()
         for name, a, b in zip(("O", "dQ", "dK", "dV"), (o, dq, dk, dv), ref):
-            assert torch.equal(a, b), name
+            if name == "dQ":
+                assert_dq_consistent(a, b)
+            else:
+                assert torch.equal(a, b), name
     finally:
         dist.destroy_process_group()
 

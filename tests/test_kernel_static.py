@@ -12,7 +12,7 @@ import re
 import pytest
 
 CSRC = pathlib.Path(__file__).resolve().parents[1] / "dynamic_block_sparse_variance_b200" / "csrc"
-SOURCES = ["attn_tc_fwd.cuh", "attn_tc_bwd.cuh", "attn_tc_bwd_fused.cuh"]
+SOURCES = ["attn_tc_fwd.cuh", "attn_tc_bwd.cuh"]
 
 
 def _kernels(text):
