@@ -538,48 +538,63 @@ __global__ void __launch_bounds__(kFbThreads, 1) bsa_bwd_tc_kernel(const __grid_
         break;
       }
       tc::tc_fence_after();
-      uint32_t lo0[16];
+      // four chunks of 16 query columns; chunk c+1's load overlaps chunk c's arithmetic
+      uint32_t dpa[16], dpb[16], lo01[8];
+      tc::tmem_ld16(colDP, dpa);
+      tc::tmem_ld_wait_regs(dpa);
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t dp[32], dk[16], lo[16];
-        tc::tmem_ld32(colDP + 32u * cc, dp);   // chunk 0's stores below land on columns already read
-        tc::tmem_ld_wait();
+      for (int c = 0; c < 4; ++c) {
+        uint32_t(&cur)[16] = (c & 1) ? dpb : dpa;
+        uint32_t(&nxt)[16] = (c & 1) ? dpa : dpb;
+        if (c < 3) tc::tmem_ld16(colDP + 16u * (c + 1), nxt);
+        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const float4 Dv = st_d[8 * cc + g];   // padding columns have P = 0, so dS = 0 there
+        for (int g = 0; g < 4; ++g) {   // four query columns at a time: 16c + 4g ..
+          const float4 Dv = st_d[4 * c + g];   // padding columns have P = 0, so dS = 0 there
+          const int j = 16 * c + 4 * g;        // column within the half
+          const uint32_t *pc = &pv[j >> 5][j & 31];
           // 2^15 dS = 2^15 P (dP - D)
-          const float2 d01 = tc::mul2(tc::f2u(pv[cc][4 * g + 0], pv[cc][4 * g + 1]),
-                                      tc::fma2(tc::f2u(dp[4 * g + 0], dp[4 * g + 1]), tc::f2(cdP, cdP), tc::f2(-Dv.x, -Dv.y)));
-          const float2 d23 = tc::mul2(tc::f2u(pv[cc][4 * g + 2], pv[cc][4 * g + 3]),
-                                      tc::fma2(tc::f2u(dp[4 * g + 2], dp[4 * g + 3]), tc::f2(cdP, cdP), tc::f2(-Dv.z, -Dv.w)));
-          dk[2 * g] = pack_bf16(d01.x, d01.y);
-          dk[2 * g + 1] = pack_bf16(d23.x, d23.y);
-          // the residuals dS - bf16(dS), exact in fp32, as the low bf16 halves
-          const float2 r01 = tc::sub2(d01, tc::f2(bf16_lo(dk[2 * g]), bf16_hi(dk[2 * g])));
-          const float2 r23 = tc::sub2(d23, tc::f2(bf16_lo(dk[2 * g + 1]), bf16_hi(dk[2 * g + 1])));
+          const float2 d01 = tc::mul2(tc::f2u(pc[0], pc[1]),
+                                      tc::fma2(tc::f2u(cur[4 * g + 0], cur[4 * g + 1]), tc::f2(cdP, cdP), tc::f2(-Dv.x, -Dv.y)));
+          const float2 d23 = tc::mul2(tc::f2u(pc[2], pc[3]),
+                                      tc::fma2(tc::f2u(cur[4 * g + 2], cur[4 * g + 3]), tc::f2(cdP, cdP), tc::f2(-Dv.z, -Dv.w)));
+          // dS_hi = dS truncated to bf16 (the top 16 bits), dS_lo = bf16(dS - dS_hi), the
+          // difference exact in fp32: about 16 significant bits together
+          const float h0 = __uint_as_float(__float_as_uint(d01.x) & 0xffff0000u);
+          const float h1 = __uint_as_float(__float_as_uint(d01.y) & 0xffff0000u);
+          const float h2 = __uint_as_float(__float_as_uint(d23.x) & 0xffff0000u);
+          const float h3 = __uint_as_float(__float_as_uint(d23.y) & 0xffff0000u);
+          hi[2 * g] = __byte_perm(__float_as_uint(d01.x), __float_as_uint(d01.y), 0x7632);
+          hi[2 * g + 1] = __byte_perm(__float_as_uint(d23.x), __float_as_uint(d23.y), 0x7632);
+          const float2 r01 = tc::sub2(d01, tc::f2(h0, h1));
+          const float2 r23 = tc::sub2(d23, tc::f2(h2, h3));
           lo[2 * g] = pack_bf16(r01.x, r01.y);
           lo[2 * g + 1] = pack_bf16(r23.x, r23.y);
         }
-        tc::tmem_st16(colDP + 16u * cc, dk);
-        // the low halves go to columns 32..63 of the range, which chunk 1's load must
-        // have read first: chunk 0's are kept until then
-        if (cc == 0) {
+        tc::tmem_st8(colDP + 8u * c, hi);   // columns already read
 #pragma unroll
-          for (int e = 0; e < 16; ++e) lo0[e] = lo[e];
-        } else {
-          tc::tmem_st16(colDP + 32u, lo0);
-          tc::tmem_st16(colDP + 48u, lo);
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {   // 16-byte chunk 4cc + c of the row: queries 8(4cc + c) .. +7
-          const int ch = 4 * cc + c;
+        for (int u = 0; u < 2; ++u) {   // 16-byte chunk 2c + u of the row: queries 8(2c + u) .. +7
+          const int ch = 2 * c + u;
           const uint32_t off = (uint32_t)((ch ^ (row & 7)) << 4);
-          const uint4 w = krow ? make_uint4(dk[4 * c], dk[4 * c + 1], dk[4 * c + 2], dk[4 * c + 3])
+          const uint4 w = krow ? make_uint4(hi[4 * u], hi[4 * u + 1], hi[4 * u + 2], hi[4 * u + 3])
                                : make_uint4(0u, 0u, 0u, 0u);
-          const uint4 wl = krow ? make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3])
+          const uint4 wl = krow ? make_uint4(lo[4 * u], lo[4 * u + 1], lo[4 * u + 2], lo[4 * u + 3])
                                 : make_uint4(0u, 0u, 0u, 0u);
           *reinterpret_cast<uint4 *>(ds_row + off) = w;
           *reinterpret_cast<uint4 *>(ds_row + kTcTileBytes + off) = wl;
+        }
+        // dS_lo^T goes to columns 32 + 8c, which chunks 2 and 3 occupy until they are read
+        if (c < 3) tc::tmem_ld_wait_regs(nxt);
+        if (c == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lo01[e] = lo[e];
+        } else if (c == 1) {   // chunk 2 has been read
+          tc::tmem_st8(colDP + 32u, lo01);
+          tc::tmem_st8(colDP + 40u, lo);
+        } else if (c == 2) {   // chunk 3 has been read
+          tc::tmem_st8(colDP + 48u, lo);
+        } else {
+          tc::tmem_st8(colDP + 56u, lo);
         }
       }
       tc::tmem_st_wait();
