@@ -133,12 +133,19 @@ KERNEL_FLOP_UNITS = {"bsa_fwd_mma_kernel": 4, "bsa_fwd_tc_kernel": 4, "bsa_fwd_t
 FWD_KERNELS = ("bsa_fwd_mma_kernel", "bsa_fwd_tc_kernel", "bsa_fwd_tc2_kernel")
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
-# kernel from one ncu capture on a smaller grid, as bytes per algorithmic FLOP
-# (the counters of a single-kernel capture on the 720p-like grid).  The full-size figure is scaled
-# by the launch's algorithmic FLOPs, and reported only while the kernel's
-# sources hash to the value they had when the counters were taken.
+# kernel from one ncu capture on a smaller grid, as bytes per algorithmic FLOP.
+# The backward's record is the 2K grid with 2 heads (the same selection
+# density and per-head working set as the 24-head grid; one launch, counters
+# dram__bytes_read.sum + dram__bytes_write.sum).  The full-size figure is
+# scaled by the launch's algorithmic FLOPs (the heads are independent
+# problems), and reported only while the kernel's sources hash to the value
+# they had when the counters were taken.
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_fwd.cuh", "tc_common.cuh", "v16.cuh")
-PROFILED_TRAFFIC = {}
+PROFILED_TRAFFIC = {
+    "bsa_bwd_tc_kernel": dict(bytes=547118283264 + 287245915648, flops=205282664775680.0,
+                              grid="2K-like with 2 heads (64x96x160)",
+                              sha256="5a0cc86e5226ec682e7e9c4b6ffe0d4cf86f9beab158d901e827a19f99e5e9e8"),
+}
 
 
 def profiled_traffic(kernel, flops_per_launch):
@@ -440,10 +447,7 @@ def run_prism(args, rank, world):
         metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
         ms_per_step=ms, higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16",
         data="synthetic",
-        config=dict(workload=f"{wl.name}-like grid {wl.T}x{wl.H}x{wl.W}", T=wl.T, H=wl.H, W=wl.W, N=wl.N,
-                    heads=wl.heads, head_dim=wl.head_dim, top_k=wl.top_k, top_p=wl.top_p,
-                    l2="inputs larger than L2 (each Q/K/V tensor %.2f GB)" % (wl.N * wl.heads * wl.head_dim * 2 / 1e9),
-                    parallelism=f"replicas x{world}"),
+        config=workload_config(wl, world),
         roofline=roof,
         attention=dict(fwd_ms=t_fwd, bwd_ms=t_bwd, executed_tflop=exec_flops / 1e12,
                        dense_equiv_tflop=dense_flops / 1e12,
@@ -525,6 +529,14 @@ def run_e2e(att, inputs, outs, wl, exec_flops, args, world):
 
 
 # ----------------------------------------------------- reference (oracle) --
+def workload_config(wl, world):
+    """The workload both arms name: grid, heads, selection knobs, L2 regime, ranks."""
+    return dict(workload=f"{wl.name}-like grid {wl.T}x{wl.H}x{wl.W}", T=wl.T, H=wl.H, W=wl.W, N=wl.N,
+                heads=wl.heads, head_dim=wl.head_dim, top_k=wl.top_k, top_p=wl.top_p,
+                l2="inputs larger than L2 (each Q/K/V tensor %.2f GB)" % (wl.N * wl.heads * wl.head_dim * 2 / 1e9),
+                parallelism=f"replicas x{world}")
+
+
 def run_reference(args, rank, world):
     """The fp64 CPU oracle on the host cores, on a bounded sample of the workload."""
     if rank != 0:
@@ -541,9 +553,7 @@ def run_reference(args, rank, world):
         metric=METRIC, value=value, unit=UNIT, n_gpus=world, steps=args.steps, warmup=args.warmup,
         ms_per_step=cb["seconds"] * 1e3 / max(1, args.steps), higher_is_better=True, scaling="weak",
         vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
-        config=dict(workload=f"{wl.name}-like grid {wl.T}x{wl.H}x{wl.W}", T=wl.T, H=wl.H, W=wl.W,
-                    heads=wl.heads, head_dim=wl.head_dim, top_k=wl.top_k, top_p=wl.top_p,
-                    parallelism="host cores"),
+        config=workload_config(wl, world),
         cpu_baseline=dict(kind="oracle", cores=cb["cores"], sample=cb["sample"], value=value, unit=UNIT),
         e2e=dict(value=value, unit=UNIT, h2d_bytes_per_step=0, d2h_bytes_per_step=0),
         gpu_launches=0,
