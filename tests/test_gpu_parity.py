@@ -19,7 +19,7 @@ from tests.helpers import (assert_close_attn, assert_dq_consistent, blocks_to_de
                            f64, selection_row_ok)
 
 pytestmark = pytest.mark.gpu
-CASES = ["tiny", "aniso8", "mix16"]
+CASES = ["tiny", "aniso8", "mix16", "smoke128"]
 _CACHE = {}
 
 
