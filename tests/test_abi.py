@@ -43,8 +43,13 @@ def test_workspace_sizes(lib):
     cap = 8 * (64 * 96 * 160 // 512)
     assert ind > 0 and sel_min >= cap * cap * 4 and sel_all >= 24 * cap * cap * 4
     assert bwd >= 4 * 10**8
-    fwd, _ = P.prism_workspace_size(p, P.PRISM_WS_FWD)
     N = 64 * 96 * 160
+    rows = 24 * N
+    # head_dim 128: fp16 copies of V and dO, the fp32 dQ accumulator, three padded per-row stats
+    assert bwd >= 10**8 * 4 + rows * 128 * (2 * 2 + 4) + 3 * (rows + 128) * 4
+    bwd64, _ = P.prism_workspace_size(P.make_params(64, 96, 160, 24, 64, 32, 0.9), P.PRISM_WS_BWD, 10**8)
+    assert bwd64 < bwd - rows * 128 * 8 // 2      # the warp-MMA backward has no copies or accumulator
+    fwd, _ = P.prism_workspace_size(p, P.PRISM_WS_FWD)
     assert 24 * N * 128 * 2 <= fwd <= 24 * N * 128 * 2 + 4096    # fp16 copy of V, per-head maxima
     p64 = P.make_params(8, 16, 16, 2, 64, 2, 0.9)
     assert P.prism_workspace_size(p64, P.PRISM_WS_FWD)[0] == 0
