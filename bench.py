@@ -144,7 +144,7 @@ ATTN_SOURCES = ("attn_common.cuh", "attn_tc_bwd.cuh", "attn_tc_fwd.cuh", "tc_com
 PROFILED_TRAFFIC = {
     "bsa_bwd_tc_kernel": dict(bytes=547118283264 + 287245915648, flops=205282664775680.0,
                               grid="2K-like with 2 heads (64x96x160)",
-                              sha256="5a0cc86e5226ec682e7e9c4b6ffe0d4cf86f9beab158d901e827a19f99e5e9e8"),
+                              sha256="dab8a993bc9c686b18e82b110934f8c4ffc15e90b3defb0551e1f6dcb315378e"),
 }
 
 

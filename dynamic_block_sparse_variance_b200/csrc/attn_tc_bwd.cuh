@@ -18,9 +18,10 @@
 //
 // Precision.  Every product accumulates in fp32 and takes its operands at the
 // precision the errors they carry allow:
-//   * P, the forward's: P_c = t(2^(x_c - m)) 2^(m - LSE), x_c the score in
-//     log2 units, m = ceil(LSE) - 15 an integer and t() truncation to 11
-//     significant bits, which is what the forward used for O = sum_c P_c v_c
+//   * P, the forward's: P_c = t(2^(x_c - m)) 2^(m - L), x_c the score and
+//     L = LSE log2e in log2 units, m = ceil(L) - 15 an integer and t()
+//     truncation to 11 significant bits, which is what the forward used for
+//     O = sum_c P_c v_c
 //     (it truncates the same way, with an integer running max, and normalises
 //     by the sum of the truncated values).  So D = rowsum(dO o O) equals
 //     sum_c P_c dP_c and every row of dS = P (dP - D) sums to zero, as it must:
@@ -32,8 +33,9 @@
 //     query row; fp16's 11 bits keep that sum's error near 2^-11 of sum |P dO|.
 //   * dP^T = V dO^T in fp16 x fp16, V likewise scaled (exact).
 //   * S^T = K Q^T, dK += dS^T Q and dQ = dS K in bf16 x bf16, the inputs
-//     themselves, with dS as the pair bf16(dS) + bf16(dS - bf16(dS)) (about
-//     16 bits, and bf16's exponent range, which the dS of key blocks that few
+//     themselves, with dS as the pair dS_hi = dS truncated to bf16 and
+//     dS_lo = bf16(dS - dS_hi) (about 16 bits together, and bf16's exponent
+//     range, which the dS of key blocks that few
 //     queries attend to need: their dS lies far below the head's largest).
 //     One rounding of dS would leave dK of heavily selected key blocks (sums
 //     over thousands of query rows) and dQ (the rows of dS sum to zero, so
