@@ -389,6 +389,10 @@ def run_prism(args, rank, world):
     unit_of = {"bsa_fwd_tc2_kernel": float(pairs256) * wl.head_dim,
                "bsa_fwd_tc_kernel": float(pairs - pairs256) * wl.head_dim}
     exec_flops = 14.0 * Punit
+    # the products the attention kernels run, in the same units: 4 P forward and 14 P backward (the
+    # tensor-core backward's second dK and dQ products on the low halves of dS, or the warp-MMA
+    # backward's recomputed S and dP), against the 14 P of the algorithm
+    product_flops = 18.0 * Punit
     dense_flops = 14.0 * float(wl.N) ** 2 * wl.head_dim * wl.heads
 
     clocks = ClockSampler(dev)
@@ -452,6 +456,8 @@ def run_prism(args, rank, world):
         attention=dict(fwd_ms=t_fwd, bwd_ms=t_bwd, executed_tflop=exec_flops / 1e12,
                        dense_equiv_tflop=dense_flops / 1e12,
                        attn_executed_tflops=exec_flops / ((t_fwd + t_bwd) * 1e-3) / 1e12 if t_fwd + t_bwd else None,
+                       product_tflop=product_flops / 1e12,
+                       attn_product_tflops=product_flops / ((t_fwd + t_bwd) * 1e-3) / 1e12 if t_fwd + t_bwd else None,
                        step_executed_pct_of_burst_peak=100.0 * exec_flops / (ms * 1e-3) / 1e12 / burst,
                        dense_equiv_tflops=dense_flops / (ms * 1e-3) / 1e12,
                        flop_density=pairs / (wl.heads * float(wl.N) ** 2),
